@@ -1,0 +1,297 @@
+"""Plain fp64 CPU oracle for training-free Top-p block-sparse video attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import this module:
+only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
+It shares no code with the CUDA library and never imports it.
+
+What it computes, step by step, and the passages each step follows:
+
+* FVAttn abstract ("video-aware block organization"): tokens of a T x Hh x W
+  latent grid are grouped into spatio-temporal cubes of ct x ch x cw tokens;
+  each cube is one block of ``bs = ct*ch*cw`` slots. ``reorder``/``unreorder``.
+* FVAttn abstract ("Top-p routing, a Top-k safety floor"): each query block
+  scores every key block with the softmax of mean-pooled Q and K blocks,
+  ``softmax_j(Qbar_i . Kbar_j / sqrt(d))``, and keeps the smallest prefix of key
+  blocks, in descending score order, whose cumulative mass reaches p, but never
+  fewer than k blocks. ``pool``, ``block_probs``, ``select_row``, ``build_mask``.
+* FVAttn abstract (the sparse attention that the mask drives): for every query
+  of block i, exact softmax attention over the keys of the selected blocks
+  only. ``attention``.
+
+Readings where the pages are silent (each listed in the design notes):
+
+* ragged grids are padded up to whole cubes; a padding slot keeps its
+  geometric place inside its cube and holds zeros;
+* cubes are ordered row-major over the cube grid (t, h, w) and tokens row-major
+  inside a cube;
+* pooled means divide by the number of valid tokens of the block;
+* no length correction of partial blocks, no forced diagonal, no causality;
+* Top-p takes the shortest prefix with cumulative mass >= p (inclusive);
+  when the floating-point sum never reaches p, or p >= 1, every block is kept;
+* ties between equal scores go to the lower key-block index;
+* k larger than the number of key blocks keeps every block;
+* padding query slots produce O = 0 and lse = 0.
+
+Parity is pinned by tests/test_oracle.py (brute force, closed forms,
+library routines, invariants); no function here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+
+@dataclass(frozen=True)
+class Geom:
+    """Grid and cube geometry (FVAttn abstract: video-aware block organization)."""
+
+    T: int
+    Hh: int
+    W: int
+    ct: int
+    ch: int
+    cw: int
+
+    @property
+    def N(self):
+        return self.T * self.Hh * self.W
+
+    @property
+    def bs(self):
+        return self.ct * self.ch * self.cw
+
+    @property
+    def nT(self):
+        return -(-self.T // self.ct)
+
+    @property
+    def nH(self):
+        return -(-self.Hh // self.ch)
+
+    @property
+    def nW(self):
+        return -(-self.W // self.cw)
+
+    @property
+    def nb(self):
+        return self.nT * self.nH * self.nW
+
+    @property
+    def Npad(self):
+        return self.nb * self.bs
+
+
+# ---------------------------------------------------------------------------
+# Video-aware block organization (FVAttn abstract)
+# ---------------------------------------------------------------------------
+
+def slot_of_token(g: Geom) -> np.ndarray:
+    """Slot of every raster token ``n = (t*Hh + h)*W + w``.
+
+    The token lands in cube ``blk = (t//ct * nH + h//ch) * nW + w//cw`` at
+    in-cube offset ``((t%ct)*ch + h%ch)*cw + w%cw``; slot = blk*bs + offset.
+    """
+    t, h, w = np.meshgrid(np.arange(g.T), np.arange(g.Hh), np.arange(g.W), indexing="ij")
+    t, h, w = t.ravel(), h.ravel(), w.ravel()
+    blk = ((t // g.ct) * g.nH + (h // g.ch)) * g.nW + (w // g.cw)
+    off = ((t % g.ct) * g.ch + (h % g.ch)) * g.cw + (w % g.cw)
+    return (blk * g.bs + off).astype(np.int64)
+
+
+def slot_of_token_loops(g: Geom) -> np.ndarray:
+    """The same permutation written as explicit loops over cubes and in-cube
+    positions (small grids only): enumerate slots in order, skip padding."""
+    out = np.full(g.N, -1, dtype=np.int64)
+    s = 0
+    for tt in range(g.nT):
+        for th in range(g.nH):
+            for tw in range(g.nW):
+                for lt in range(g.ct):
+                    for lh in range(g.ch):
+                        for lw in range(g.cw):
+                            t, h, w = tt * g.ct + lt, th * g.ch + lh, tw * g.cw + lw
+                            if t < g.T and h < g.Hh and w < g.W:
+                                out[(t * g.Hh + h) * g.W + w] = s
+                            s += 1
+    return out
+
+
+def slot_valid(g: Geom) -> np.ndarray:
+    """Boolean [Npad]: True where the slot holds a real token."""
+    v = np.zeros(g.Npad, dtype=bool)
+    v[slot_of_token(g)] = True
+    return v
+
+
+def block_len(g: Geom) -> np.ndarray:
+    """Number of real tokens in every block, by counting valid slots."""
+    return slot_valid(g).reshape(g.nb, g.bs).sum(axis=1).astype(np.int64)
+
+
+def reorder(X: np.ndarray, g: Geom) -> np.ndarray:
+    """[B,H,N,d] raster -> [B,H,Npad,d] cube order, padding slots zero (fp64)."""
+    B, H, N, d = X.shape
+    assert N == g.N
+    Xt = np.zeros((B, H, g.Npad, d), dtype=np.float64)
+    Xt[:, :, slot_of_token(g)] = X
+    return Xt
+
+
+def unreorder(Xt: np.ndarray, g: Geom) -> np.ndarray:
+    """[B,H,Npad,d] cube order -> [B,H,N,d] raster; padding slots are dropped."""
+    return np.asarray(Xt, dtype=np.float64)[:, :, slot_of_token(g)]
+
+
+# ---------------------------------------------------------------------------
+# Block scoring and Top-p / Top-k routing (FVAttn abstract)
+# ---------------------------------------------------------------------------
+
+def pool(Xt: np.ndarray, g: Geom) -> np.ndarray:
+    """Mean of the real tokens of every block: [B,H,Npad,d] -> [B,H,nb,d]."""
+    B, H, _, d = Xt.shape
+    valid = slot_valid(g).reshape(g.nb, g.bs)
+    blocks = np.asarray(Xt, dtype=np.float64).reshape(B, H, g.nb, g.bs, d)
+    sums = (blocks * valid[None, None, :, :, None]).sum(axis=3)
+    return sums / block_len(g)[None, None, :, None]
+
+
+def block_probs(Qbar: np.ndarray, Kbar: np.ndarray) -> np.ndarray:
+    """Row softmax over key blocks of ``Qbar Kbar^T / sqrt(d)``: [..,nb,d] -> [..,nb,nb]."""
+    d = Qbar.shape[-1]
+    S = np.matmul(Qbar, np.swapaxes(Kbar, -1, -2)) / math.sqrt(d)
+    S = S - S.max(axis=-1, keepdims=True)
+    E = np.exp(S)
+    return E / E.sum(axis=-1, keepdims=True)
+
+
+def select_row(P: np.ndarray, p: float, k: int):
+    """Top-p with a Top-k floor on one row of block probabilities.
+
+    Sort descending (ties: lower index first), take the shortest prefix whose
+    cumulative mass reaches p, then at least k entries, at most all of them.
+    Returns (selected indices ascending, info) where info carries the
+    quantities the exemption rules need.
+    """
+    P = np.asarray(P, dtype=np.float64)
+    nkb = P.shape[0]
+    order = np.lexsort((np.arange(nkb), -P))
+    c = np.cumsum(P[order])
+    if p >= 1.0:
+        n_p = nkb
+    else:
+        hit = np.nonzero(c >= p)[0]
+        n_p = int(hit[0]) + 1 if hit.size else nkb
+    n = min(nkb, max(int(k), n_p))
+    sel = np.sort(order[:n])
+    info = {
+        "n_p": n_p,
+        "n": n,
+        "c_at": float(c[n_p - 1]),
+        "c_before": float(c[n_p - 2]) if n_p >= 2 else 0.0,
+        "gap": float(P[order[n - 1]] - P[order[n]]) if n < nkb else math.inf,
+        "order": order,
+    }
+    return sel, info
+
+
+def build_mask(Qt: np.ndarray, Kt: np.ndarray, g: Geom, top_p, top_k: int,
+               boundary_tol: float = 1e-4, tie_tol: float = 1e-6) -> dict:
+    """Pool, score, select every (b, h, query block) row; emit bitmask and CSR.
+
+    Rows are flattened as r = (b*H + h)*nb + i. ``col_idx`` is ascending inside
+    each row. Bit j of a row lives in word j//32 at position j%32.
+    ``boundary`` marks rows whose cumulative mass at the cut lies within
+    ``boundary_tol`` of p; ``near_tie`` rows whose last kept and first dropped
+    probabilities differ by at most ``tie_tol``.
+    """
+    B, H = Qt.shape[:2]
+    nb = g.nb
+    words = -(-nb // 32)
+    Pm = block_probs(pool(Qt, g), pool(Kt, g))  # [B,H,nb,nb]
+    R = B * H * nb
+    row_cnt = np.zeros(R, dtype=np.int64)
+    bitmask = np.zeros((R, words), dtype=np.uint32)
+    boundary = np.zeros(R, dtype=bool)
+    near_tie = np.zeros(R, dtype=bool)
+    cols = []
+    for b in range(B):
+        for h in range(H):
+            p = float(top_p[h])
+            for i in range(nb):
+                r = (b * H + h) * nb + i
+                sel, info = select_row(Pm[b, h, i], p, top_k)
+                row_cnt[r] = sel.size
+                cols.append(sel)
+                for j in sel:
+                    bitmask[r, j // 32] |= np.uint32(1 << (j % 32))
+                boundary[r] = (abs(info["c_at"] - p) <= boundary_tol
+                               or abs(info["c_before"] - p) <= boundary_tol)
+                near_tie[r] = info["gap"] <= tie_tol
+    row_ptr = np.zeros(R + 1, dtype=np.int64)
+    row_ptr[1:] = np.cumsum(row_cnt)
+    col_idx = np.concatenate(cols).astype(np.int64) if cols else np.zeros(0, np.int64)
+    return {"probs": Pm, "row_cnt": row_cnt, "row_ptr": row_ptr, "col_idx": col_idx,
+            "bitmask": bitmask, "boundary": boundary, "near_tie": near_tie}
+
+
+def lpt_order(row_cnt: np.ndarray) -> np.ndarray:
+    """Work order, longest first: rows by selected-block count descending,
+    equal counts by row index ascending (FVAttn abstract: uneven per-head
+    workloads; scheduling the heaviest rows first limits the straggler tail)."""
+    row_cnt = np.asarray(row_cnt)
+    return np.lexsort((np.arange(row_cnt.size), -row_cnt)).astype(np.int64)
+
+
+# ---------------------------------------------------------------------------
+# Block-sparse attention (FVAttn abstract)
+# ---------------------------------------------------------------------------
+
+def attention(Qt, Kt, Vt, g: Geom, row_ptr, col_idx, blocks=None):
+    """Exact softmax attention of every real query slot over the real key slots
+    of its block's selected key blocks.
+
+    ``blocks``: optional iterable of (b, h, i) query blocks to compute; others
+    are left NaN. Returns (Ot [B,H,Npad,d], lse [B,H,Npad]) in fp64 where
+    ``lse = log sum_k exp(q.k / sqrt(d))`` (natural log). Padding query slots
+    give O = 0 and lse = 0.
+    """
+    Qt = np.asarray(Qt, dtype=np.float64)
+    Kt = np.asarray(Kt, dtype=np.float64)
+    Vt = np.asarray(Vt, dtype=np.float64)
+    B, H, Npad, d = Qt.shape
+    nb, bs = g.nb, g.bs
+    valid = slot_valid(g)
+    Ot = np.full((B, H, Npad, d), np.nan)
+    lse = np.full((B, H, Npad), np.nan)
+    if blocks is None:
+        blocks = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
+    scale = 1.0 / math.sqrt(d)
+    for (b, h, i) in blocks:
+        r = (b * H + h) * nb + i
+        sel = np.asarray(col_idx[row_ptr[r]:row_ptr[r + 1]], dtype=np.int64)
+        key_slots = (sel[:, None] * bs + np.arange(bs)[None, :]).ravel()
+        key_slots = key_slots[valid[key_slots]]
+        q_slots = np.arange(i * bs, (i + 1) * bs)
+        q = Qt[b, h, q_slots]
+        s = (q @ Kt[b, h, key_slots].T) * scale
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        l = e.sum(axis=1, keepdims=True)
+        o = (e / l) @ Vt[b, h, key_slots]
+        qv = valid[q_slots]
+        o[~qv] = 0.0
+        ls = (m + np.log(l))[:, 0]
+        ls[~qv] = 0.0
+        Ot[b, h, q_slots] = o
+        lse[b, h, q_slots] = ls
+    return Ot, lse
+
+
+def forward(q, k, v, g: Geom, top_p, top_k: int):
+    """The whole path on raster inputs: reorder, route, attend, unreorder."""
+    qt, kt, vt = reorder(q, g), reorder(k, g), reorder(v, g)
+    m = build_mask(qt, kt, g, top_p, top_k)
+    ot, lse = attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"])
+    return unreorder(ot, g), m, lse

@@ -1,0 +1,375 @@
+"""Pins for the fp64 oracle against things other than itself: hand-worked
+examples, brute force over tiny inputs, closed forms, library routines and
+invariants. CPU only.
+
+Each group names the plausible mistake it is there to catch.
+"""
+import itertools
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+from oracle import Geom
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+GEOMS = [
+    Geom(4, 8, 8, 4, 4, 4),      # tiny workload grid (divisible)
+    Geom(8, 16, 16, 4, 4, 4),    # small workload grid (divisible)
+    Geom(5, 9, 7, 2, 4, 4),      # ragged in every axis
+    Geom(3, 3, 3, 2, 2, 2),
+    Geom(1, 1, 1, 1, 1, 1),
+    Geom(2, 3, 3, 1, 2, 2),
+    Geom(21, 30, 52, 2, 8, 8),   # Wan-shaped grid (ragged t, h, w)
+]
+
+
+# ----------------------------------------------------------------- permutation
+# catches: swapped axes, wrong cube-grid strides, wrong in-cube order
+
+@pytest.mark.parametrize("g", GEOMS, ids=str)
+def test_perm_formula_matches_explicit_loops(g):
+    assert np.array_equal(oracle.slot_of_token(g), oracle.slot_of_token_loops(g))
+
+
+def test_perm_hand_worked_example():
+    lines = [l for l in open(os.path.join(GOLDEN, "perm_worked.txt")) if not l.startswith("#")]
+    kv = {l.split(":")[0]: [int(x) for x in l.split(":")[1].split()] for l in lines if ":" in l}
+    g = Geom(*kv["geometry"])
+    assert oracle.slot_of_token(g).tolist() == kv["slot_of_token"]
+    assert oracle.block_len(g).tolist() == kv["block_len"]
+
+
+@pytest.mark.parametrize("g", [Geom(4, 8, 8, 4, 4, 4), Geom(8, 16, 16, 4, 4, 4),
+                               Geom(4, 16, 24, 2, 8, 8)], ids=str)
+def test_perm_divisible_grid_is_a_6d_transpose(g):
+    """With no padding the cube order is the textbook reshape/transpose."""
+    rng = np.random.default_rng(1)
+    d = 3
+    X = rng.standard_normal((1, 1, g.N, d))
+    ref = (X.reshape(g.nT, g.ct, g.nH, g.ch, g.nW, g.cw, d)
+           .transpose(0, 2, 4, 1, 3, 5, 6).reshape(1, 1, g.Npad, d))
+    assert np.array_equal(oracle.reorder(X, g), ref)
+
+
+@pytest.mark.parametrize("g", GEOMS, ids=str)
+def test_perm_is_injective_onto_valid_slots_and_cubes_are_boxes(g):
+    s = oracle.slot_of_token(g)
+    assert np.unique(s).size == g.N and s.min() >= 0 and s.max() < g.Npad
+    valid = oracle.slot_valid(g)
+    assert valid.sum() == g.N and np.array_equal(np.nonzero(valid)[0], np.sort(s))
+    t, h, w = np.unravel_index(np.arange(g.N), (g.T, g.Hh, g.W))
+    blk = s // g.bs
+    for b in np.unique(blk):
+        m = blk == b
+        for c, e in ((t[m], g.ct), (h[m], g.ch), (w[m], g.cw)):
+            assert c.min() // e == c.max() // e  # one aligned box per block
+    # closed form for block lengths: product of per-axis clipped extents
+    L = oracle.block_len(g).reshape(g.nT, g.nH, g.nW)
+    for tt, th, tw in itertools.product(range(g.nT), range(g.nH), range(g.nW)):
+        exp = (min(g.ct, g.T - tt * g.ct) * min(g.ch, g.Hh - th * g.ch)
+               * min(g.cw, g.W - tw * g.cw))
+        assert L[tt, th, tw] == exp
+    assert L.sum() == g.N
+
+
+@pytest.mark.parametrize("g", GEOMS[:6], ids=str)
+def test_reorder_round_trip_and_zero_padding(g):
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((2, 3, g.N, 5))
+    Xt = oracle.reorder(X, g)
+    assert np.array_equal(oracle.unreorder(Xt, g), X)
+    assert np.all(Xt[:, :, ~oracle.slot_valid(g)] == 0)
+
+
+# --------------------------------------------------------------------- pooling
+# catches: dividing by bs instead of the valid count, pooling padding slots
+
+@pytest.mark.parametrize("g", GEOMS[:6], ids=str)
+def test_pool_of_blockwise_constant_field_is_that_constant(g):
+    rng = np.random.default_rng(3)
+    d = 4
+    C = rng.standard_normal((1, 2, g.nb, d))
+    blk = oracle.slot_of_token(g) // g.bs
+    X = C[:, :, blk]  # raster field constant on every cube
+    Qbar = oracle.pool(oracle.reorder(X, g), g)
+    np.testing.assert_allclose(Qbar, C, rtol=0, atol=1e-12)
+
+
+def test_pool_matches_explicit_mean_over_tokens():
+    g = Geom(5, 9, 7, 2, 4, 4)
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((1, 1, g.N, 3))
+    blk = oracle.slot_of_token(g) // g.bs
+    Qbar = oracle.pool(oracle.reorder(X, g), g)
+    for b in range(g.nb):
+        np.testing.assert_allclose(Qbar[0, 0, b], X[0, 0, blk == b].mean(axis=0), atol=1e-13)
+
+
+# --------------------------------------------------------------- block softmax
+# catches: wrong 1/sqrt(d) scale, transposed product, missing max shift
+
+def test_block_probs_matches_scipy_softmax():
+    rng = np.random.default_rng(5)
+    Qb = rng.standard_normal((2, 3, 11, 16)) * 3
+    Kb = rng.standard_normal((2, 3, 11, 16)) * 3
+    P = oracle.block_probs(Qb, Kb)
+    S = np.einsum("bhid,bhjd->bhij", Qb, Kb) / 4.0
+    np.testing.assert_allclose(P, scipy.special.softmax(S, axis=-1), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(P.sum(-1), 1.0, atol=1e-12)
+
+
+def test_block_probs_closed_form_scale():
+    d = 9
+    a = 2.0
+    b = np.array([0.0, 1.0, 3.0, -1.5])
+    Qb = np.zeros((1, d)); Qb[0, 0] = a
+    Kb = np.zeros((4, d)); Kb[:, 0] = b
+    # a single query row against four key rows: exp(a*b_j/3) / sum
+    P = oracle.block_probs(Qb, Kb)[0]
+    e = np.exp(a * b / 3.0)
+    np.testing.assert_allclose(P, e / e.sum(), rtol=1e-14)
+    # asymmetric rows: P[i, j] uses Q row i and K row j, not the transpose
+    Qb2 = np.stack([Qb[0], 2 * Qb[0]])
+    P2 = oracle.block_probs(Qb2, Kb[:2])
+    e2 = np.exp(2 * a * b[:2] / 3.0)
+    np.testing.assert_allclose(P2[1], e2 / e2.sum(), rtol=1e-14)
+
+
+def test_block_probs_survive_huge_scores():
+    Qb = np.array([[800.0, 0.0]])
+    Kb = np.array([[1.0, 0.0], [0.9, 0.0]])
+    P = oracle.block_probs(Qb, Kb)
+    assert np.all(np.isfinite(P)) and abs(P.sum() - 1) < 1e-12
+
+
+# ------------------------------------------------------------------- selection
+# catches: exclusive instead of inclusive cut, wrong tie order, floor ignored
+
+def _golden_rows():
+    for line in open(os.path.join(GOLDEN, "select_worked.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        probs, p, k, exp = [x.strip() for x in line.split("|")]
+        yield ([float(x) for x in probs.split(",")], float(p), int(k),
+               [int(x) for x in exp.split(",")])
+
+
+@pytest.mark.parametrize("probs,p,k,exp", list(_golden_rows()))
+def test_select_hand_worked(probs, p, k, exp):
+    sel, _ = oracle.select_row(np.array(probs), p, k)
+    assert sel.tolist() == exp
+
+
+def _brute_force_select(P_frac, p_frac, k):
+    """Exact (rational) brute force over every subset: the smallest subset
+    size whose best subset reaches mass p, floored at k and capped at nkb;
+    among the heaviest subsets of that size the lexicographically smallest
+    index tuple (the lower-index tie rule)."""
+    nkb = len(P_frac)
+    n_p = nkb
+    for n in range(1, nkb + 1):
+        best = max(sum(P_frac[j] for j in c) for c in itertools.combinations(range(nkb), n))
+        if best >= p_frac:
+            n_p = n
+            break
+    n = min(nkb, max(k, n_p))
+    cands = list(itertools.combinations(range(nkb), n))
+    best = max(sum(P_frac[j] for j in c) for c in cands)
+    return min(c for c in cands if sum(P_frac[j] for j in c) == best)
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_select_matches_brute_force_over_subsets(seed):
+    rng = np.random.default_rng(100 + seed)
+    nkb = int(rng.integers(1, 10))
+    # dyadic probabilities: integers over 64, frequent ties, exact sums
+    w = rng.integers(0, 6, size=nkb) if seed % 3 else rng.integers(0, 3, size=nkb)
+    if w.sum() == 0:
+        w[0] = 1
+    denom = 1 << 10
+    raw = (w * (denom // w.sum())).astype(np.int64)
+    raw[0] += denom - raw.sum()
+    if raw[0] < 0:
+        return
+    P_frac = [Fraction(int(x), denom) for x in raw]
+    p_frac = Fraction(int(rng.integers(1, denom + 1)), denom)
+    k = int(rng.integers(0, nkb + 2))
+    sel, _ = oracle.select_row(np.array([float(x) for x in P_frac]), float(p_frac), k)
+    assert tuple(sel.tolist()) == _brute_force_select(P_frac, p_frac, k)
+
+
+def test_select_special_cases():
+    rng = np.random.default_rng(7)
+    P = scipy.special.softmax(rng.standard_normal(50) * 2)
+    assert oracle.select_row(P, 1.0, 1)[0].size == 50          # p = 1 keeps all
+    for k in (1, 3, 7):
+        sel, _ = oracle.select_row(P, 1e-12, k)                 # p -> 0: exactly top k
+        assert sel.tolist() == sorted(np.argsort(-P, kind="stable")[:k].tolist())
+    assert oracle.select_row(P, 0.5, 80)[0].size == 50         # k > nkb caps
+
+
+def _mask_invariants(m, top_p, top_k, nb):
+    R = m["row_cnt"].size
+    assert np.array_equal(m["row_ptr"][1:] - m["row_ptr"][:-1], m["row_cnt"])
+    assert m["row_ptr"][0] == 0 and np.all(np.diff(m["row_ptr"]) >= 0)
+    P = m["probs"].reshape(R, nb)
+    H = len(top_p)
+    for r in range(R):
+        cols = m["col_idx"][m["row_ptr"][r]:m["row_ptr"][r + 1]]
+        assert np.all(np.diff(cols) > 0)
+        bits = [j for j in range(nb) if (m["bitmask"][r, j // 32] >> (j % 32)) & 1]
+        assert bits == cols.tolist()
+        p = top_p[(r // nb) % H]
+        assert cols.size >= min(top_k, nb)
+        mass = P[r, cols].sum()
+        assert mass >= p - 1e-12 or cols.size == nb
+        if cols.size > max(top_k, 1):          # minimality of the Top-p prefix
+            assert mass - P[r, cols].min() < p + 1e-12
+
+
+def test_build_mask_invariants_ragged():
+    g = Geom(5, 9, 7, 2, 4, 4)
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((2, 3, g.N, 8)) * 2
+    k = rng.standard_normal((2, 3, g.N, 8)) * 2
+    top_p = [0.5, 0.8, 0.95]
+    m = oracle.build_mask(oracle.reorder(q, g), oracle.reorder(k, g), g, top_p, 2)
+    _mask_invariants(m, top_p, 2, g.nb)
+
+
+def test_lpt_order_matches_python_sort():
+    rng = np.random.default_rng(9)
+    cnt = rng.integers(0, 12, size=500)
+    exp = sorted(range(500), key=lambda r: (-cnt[r], r))
+    assert oracle.lpt_order(cnt).tolist() == exp
+
+
+# ------------------------------------------------------------------- attention
+# catches: padding keys not masked, transposed Q/K, wrong scale, padding rows
+
+def _dense_sdpa(qt, kt, vt, g):
+    """torch scaled_dot_product_attention in fp64 with a key-padding mask."""
+    valid = torch.from_numpy(oracle.slot_valid(g))
+    mask = valid[None, None, None, :].expand(qt.shape[0], qt.shape[1], qt.shape[2], -1)
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(qt), torch.from_numpy(kt), torch.from_numpy(vt), attn_mask=mask).numpy()
+
+
+@pytest.mark.parametrize("g", [Geom(5, 9, 7, 2, 4, 4), Geom(4, 8, 8, 4, 4, 4)], ids=str)
+def test_attention_p1_equals_dense_sdpa(g):
+    rng = np.random.default_rng(10)
+    q, k, v = (rng.standard_normal((1, 2, g.N, 16)) * s for s in (1.5, 1.5, 1.0))
+    qt, kt, vt = (oracle.reorder(x, g) for x in (q, k, v))
+    m = oracle.build_mask(qt, kt, g, [1.0, 1.0], 1)
+    assert np.all(m["row_cnt"] == g.nb)
+    Ot, lse = oracle.attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"])
+    ref = _dense_sdpa(qt, kt, vt, g)
+    valid = oracle.slot_valid(g)
+    np.testing.assert_allclose(Ot[:, :, valid], ref[:, :, valid], atol=1e-12, rtol=1e-10)
+    assert np.all(Ot[:, :, ~valid] == 0)
+    S = np.einsum("bhqd,bhkd->bhqk", qt, kt) / 4.0
+    S[..., ~valid] = -np.inf
+    np.testing.assert_allclose(lse[:, :, valid], scipy.special.logsumexp(S, axis=-1)[:, :, valid],
+                               atol=1e-12)
+
+
+def test_attention_closed_form_two_keys():
+    # d = 2, q = (sqrt2 ln3, 0), keys e0 and e1: weights 3/4 and 1/4, lse = ln 4
+    g = Geom(1, 1, 2, 1, 1, 2)
+    qt = np.zeros((1, 1, 2, 2)); qt[0, 0, 0, 0] = math.sqrt(2) * math.log(3)
+    kt = np.array([[[[1.0, 0.0], [0.0, 1.0]]]])
+    vt = np.array([[[[1.0, 0.0], [0.0, 1.0]]]])
+    Ot, lse = oracle.attention(qt, kt, vt, g, np.array([0, 1]), np.array([0]))
+    np.testing.assert_allclose(Ot[0, 0, 0], [0.75, 0.25], atol=1e-15)
+    np.testing.assert_allclose(lse[0, 0, 0], math.log(4), atol=1e-15)
+
+
+def test_attention_explicit_loops_on_sparse_mask():
+    g = Geom(3, 3, 3, 2, 2, 2)
+    rng = np.random.default_rng(11)
+    q, k, v = (rng.standard_normal((1, 1, g.N, 4)) for _ in range(3))
+    qt, kt, vt = (oracle.reorder(x, g) for x in (q, k, v))
+    m = oracle.build_mask(qt, kt, g, [0.6], 2)
+    assert m["row_cnt"].min() < g.nb  # really sparse
+    Ot, lse = oracle.attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"])
+    valid = oracle.slot_valid(g)
+    for i in range(g.nb):
+        sel = m["col_idx"][m["row_ptr"][i]:m["row_ptr"][i + 1]]
+        for a in range(i * g.bs, (i + 1) * g.bs):
+            if not valid[a]:
+                continue
+            num = np.zeros(4)
+            den = 0.0
+            for j in sel:
+                for c in range(j * g.bs, (j + 1) * g.bs):
+                    if valid[c]:
+                        wgt = math.exp(sum(qt[0, 0, a, x] * kt[0, 0, c, x] for x in range(4)) / 2.0)
+                        num += wgt * vt[0, 0, c]
+                        den += wgt
+            np.testing.assert_allclose(Ot[0, 0, a], num / den, atol=1e-12)
+            np.testing.assert_allclose(lse[0, 0, a], math.log(den), atol=1e-12)
+
+
+def test_attention_rows_are_convex_combinations_and_constant_v():
+    g = Geom(5, 9, 7, 2, 4, 4)
+    rng = np.random.default_rng(12)
+    q, k = (rng.standard_normal((1, 2, g.N, 8)) * 2 for _ in range(2))
+    v = rng.standard_normal((1, 2, g.N, 8))
+    qt, kt, vt = (oracle.reorder(x, g) for x in (q, k, v))
+    m = oracle.build_mask(qt, kt, g, [0.7, 0.9], 1)
+    Ot, _ = oracle.attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"])
+    valid = oracle.slot_valid(g)
+    for h in range(2):
+        for i in range(g.nb):
+            r = h * g.nb + i
+            sel = m["col_idx"][m["row_ptr"][r]:m["row_ptr"][r + 1]]
+            ks = np.concatenate([np.arange(j * g.bs, (j + 1) * g.bs) for j in sel])
+            ks = ks[valid[ks]]
+            lo, hi = vt[0, h, ks].min(0), vt[0, h, ks].max(0)
+            for a in range(i * g.bs, (i + 1) * g.bs):
+                if valid[a]:
+                    assert np.all(Ot[0, h, a] >= lo - 1e-12) and np.all(Ot[0, h, a] <= hi + 1e-12)
+    vconst = np.broadcast_to(np.arange(8.0), v.shape).copy()
+    Oc, _ = oracle.attention(qt, kt, oracle.reorder(vconst, g), g, m["row_ptr"], m["col_idx"])
+    np.testing.assert_allclose(Oc[:, :, valid], np.broadcast_to(np.arange(8.0), Oc[:, :, valid].shape),
+                               atol=1e-12)
+
+
+def test_attention_single_valid_key_returns_its_value():
+    g = Geom(1, 1, 3, 1, 1, 2)  # block 1 holds one real token (w = 2)
+    rng = np.random.default_rng(13)
+    qt, kt, vt = (oracle.reorder(rng.standard_normal((1, 1, 3, 4)), g) for _ in range(3))
+    Ot, _ = oracle.attention(qt, kt, vt, g, np.array([0, 1, 2]), np.array([1, 1]))
+    np.testing.assert_allclose(Ot[0, 0, 0], vt[0, 0, 2], atol=1e-15)
+    np.testing.assert_allclose(Ot[0, 0, 2], vt[0, 0, 2], atol=1e-15)
+
+
+def test_attention_invariant_to_key_order_inside_a_block():
+    g = Geom(4, 8, 8, 4, 4, 4)
+    rng = np.random.default_rng(14)
+    qt, kt, vt = (oracle.reorder(rng.standard_normal((1, 1, g.N, 8)), g) for _ in range(3))
+    m = oracle.build_mask(qt, kt, g, [0.8], 1)
+    O1, l1 = oracle.attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"])
+    perm = np.concatenate([j * g.bs + rng.permutation(g.bs) for j in range(g.nb)])
+    O2, l2 = oracle.attention(qt, kt[:, :, perm], vt[:, :, perm], g, m["row_ptr"], m["col_idx"])
+    np.testing.assert_allclose(O1, O2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+
+
+# ------------------------------------------------------------------ end to end
+
+def test_forward_on_tiny_workload_is_consistent():
+    import datagen
+    wl = datagen.WORKLOADS["tiny"]
+    q, k, v = (x.double().numpy() for x in datagen.generate(wl))
+    g = Geom(wl.T, wl.Hh, wl.W, *wl.cube)
+    o, m, lse = oracle.forward(q, k, v, g, wl.top_p_per_head(), wl.top_k)
+    assert o.shape == q.shape and np.all(np.isfinite(o))
+    _mask_invariants(m, wl.top_p_per_head(), wl.top_k, g.nb)
