@@ -224,8 +224,9 @@ def build_mask(Qt: np.ndarray, Kt: np.ndarray, g: Geom, top_p, top_k: int,
                 sel, info = select_row(Pm[b, h, i], p, top_k)
                 row_cnt[r] = sel.size
                 cols.append(sel)
-                for j in sel:
-                    bitmask[r, j // 32] |= np.uint32(1 << (j % 32))
+                bits = np.zeros(words * 32, dtype=bool)
+                bits[sel] = True  # bit j%32 of word j//32, least significant first
+                bitmask[r] = np.packbits(bits, bitorder="little").view("<u4")
                 boundary[r] = (abs(info["c_at"] - p) <= boundary_tol
                                or abs(info["c_before"] - p) <= boundary_tol)
                 near_tie[r] = info["gap"] <= tie_tol
