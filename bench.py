@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention hot path on B200.
+
+One step = the whole path on one batch: sba_reorder (q, k, v) ->
+sba_build_mask -> sba_attention -> sba_unreorder, on the Wan-2.1-14B-480p
+shaped layer (B=1, H=40, 21x30x52 latent grid = 32760 tokens, d=128, cubes
+2x8x8, Top-p 0.9, Top-k 8, bf16, seeded synthetic Q/K/V).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline metric: effective TFLOPS over the selected blocks, F_tile = sum over
+selected (row, key block) pairs of 4*bs^2*d, divided by the device time of a
+whole step (all four calls). Under torchrun every rank runs its own replica of
+the workload (weak scaling, no data-path collective); the time is the max over
+ranks. `--impl reference` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn effective TFLOPS (selected blocks) & % BF16 peak; ms/call"
+UNIT = "TFLOPS"
+WORKLOAD = "wan"
+L2_NOTE = "inputs (1.0 GB q/k/v) larger than the 126 MB L2, and L2 flushed by a 256 MiB write before every step (outside the timed events)"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _config(wl, extra=None):
+    cfg = {"workload": f"{wl.name}: B={wl.B} H={wl.H} grid {wl.T}x{wl.Hh}x{wl.W} "
+                       f"({wl.N} tokens) d={wl.d} cube {'x'.join(map(str, wl.cube))} "
+                       f"top_p={','.join(str(p) for p in sorted(set(wl.top_p)))} top_k={wl.top_k}",
+           "global_batch": wl.B, "seq_len": wl.N, "heads": wl.H, "head_dim": wl.d,
+           "parallelism": "replicas", "l2": L2_NOTE}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def _block_lens(wl):
+    """Real tokens per block (for the valid-FLOP count), row-major over cubes."""
+    ct, ch, cw = wl.cube
+    nT, nH, nW = -(-wl.T // ct), -(-wl.Hh // ch), -(-wl.W // cw)
+    lens = []
+    for tt in range(nT):
+        for th in range(nH):
+            for tw in range(nW):
+                lens.append(min(ct, wl.T - tt * ct) * min(ch, wl.Hh - th * ch) * min(cw, wl.W - tw * cw))
+    return lens
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0) or 0), float(d["hbm_gbs"]), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _traffic_from_profile(kernel_src: str):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "attn_sm100_wan.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"source sha256:\s*([0-9a-f]{16,64})", text)
+    m_bytes = re.search(r"dram bytes per launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes:
+        return None
+    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    if not cur.startswith(m_hash.group(1)):
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _cpu_cores():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    threads = n
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            threads = max(info)
+    except Exception:
+        pass
+    return n, threads
+
+
+def cpu_oracle_sample(wl, q, k, v, heads=(0,), blocks_per_head=None, seed=0):
+    """Time the fp64 oracle (reorder, routing, attention) on a bounded sample:
+    the given heads in full (routing) and `blocks_per_head` query blocks of
+    each (attention; all blocks when None). Returns (selected tile FLOPs,
+    seconds, description)."""
+    import numpy as np
+
+    import oracle
+    g = oracle.Geom(wl.T, wl.Hh, wl.W, *wl.cube)
+    tp = wl.top_p_per_head()
+    flops = 0.0
+    secs = 0.0
+    rng = np.random.default_rng(seed)
+    for h in heads:
+        Q, K, V = (x[:, h:h + 1].double().cpu().numpy() for x in (q, k, v))
+        t0 = time.perf_counter()
+        qt, kt, vt = oracle.reorder(Q, g), oracle.reorder(K, g), oracle.reorder(V, g)
+        m = oracle.build_mask(qt, kt, g, [tp[h]], wl.top_k)
+        if blocks_per_head is None:
+            blocks = [(0, 0, i) for i in range(g.nb)]
+        else:
+            blocks = [(0, 0, int(i)) for i in rng.choice(g.nb, size=blocks_per_head, replace=False)]
+        oracle.attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"], blocks=blocks)
+        secs += time.perf_counter() - t0
+        flops += sum(int(m["row_cnt"][i]) for (_, _, i) in blocks) * 4.0 * g.bs * g.bs * wl.d
+    nb = len(blocks)
+    desc = (f"{len(heads)} head(s) of {wl.H}: reorder + routing of the whole head, attention on "
+            f"{nb} of {g.nb} query blocks; fp64 numpy")
+    return flops, secs, desc
+
+
+def run_reference(args):
+    ws, rank, local = _dist()
+    if rank != 0:
+        return 0
+    import datagen
+    wl = datagen.WORKLOADS[args.workload]
+    q, k, v = datagen.generate(wl, seed=0, device="cpu")
+    cores, threads = _cpu_cores()
+    times, flops_tot = [], 0.0
+    desc = ""
+    for s in range(args.warmup + args.steps):
+        f, sec, desc = cpu_oracle_sample(wl, q, k, v, heads=(s % wl.H,), blocks_per_head=8, seed=s)
+        if s >= args.warmup:
+            times.append(sec)
+            flops_tot += f
+    tot = sum(times)
+    value = flops_tot / tot / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    import block_sparse_attention_sba_b200 as sba
+    import datagen
+
+    ws, rank, local = _dist()
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    wl = datagen.WORKLOADS[args.workload]
+    q, k, v = datagen.generate(wl, seed=0, device=dev)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    sa = sba.SparseAttention(plan, device=dev)
+    h = plan.handle
+    o = torch.empty_like(q)
+    top_p = wl.top_p_per_head()
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt, stream)
+        if ev:
+            ev[1].record(stream)
+        sba.sba_build_mask(h, sa.qt, sa.kt, top_p, wl.top_k, sa.bitmask, sa.row_cnt, sa.row_ptr,
+                           sa.col_idx, sa.work_order, sa.workspace, stream)
+        if ev:
+            ev[2].record(stream)
+        sba.sba_attention(h, sa.qt, sa.kt, sa.vt, sa.row_ptr, sa.col_idx, sa.work_order, sa.ot,
+                          sa.lse, sba.SBA_SCHED_LPT, None, sa.workspace, stream)
+        if ev:
+            ev[3].record(stream)
+        sba.sba_unreorder(h, sa.ot, o, stream)
+        if ev:
+            ev[4].record(stream)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    status = sa.check(stream)
+    if status != 0:
+        print(json.dumps({"error": f"device status {sba.sba_status_string(status)}"}))
+        return 1
+
+    gpu_id = str(local)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)  # let the sampler start before the timed region
+    for s in range(args.steps):
+        flush.zero_()
+        step(evs[s])
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop()
+    per_call = {"reorder": [], "build_mask": [], "attention": [], "unreorder": []}
+    step_ms = []
+    for e in evs:
+        per_call["reorder"].append(e[0].elapsed_time(e[1]))
+        per_call["build_mask"].append(e[1].elapsed_time(e[2]))
+        per_call["attention"].append(e[2].elapsed_time(e[3]))
+        per_call["unreorder"].append(e[3].elapsed_time(e[4]))
+        step_ms.append(e[0].elapsed_time(e[4]))
+    mean_step = sum(step_ms) / len(step_ms)
+    if pg:
+        t = torch.tensor([mean_step], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        mean_step = float(t.item())
+    status = sa.check(stream)
+
+    # selected-block FLOPs of one step
+    rc = sa.row_cnt.cpu().tolist()
+    cols = sa.col_idx[: int(sa.row_ptr[-1].item())].cpu().tolist()
+    rp = sa.row_ptr.cpu().tolist()
+    bs = plan.info.bs
+    nnz = rp[-1]
+    f_tile = 4.0 * bs * bs * wl.d * nnz
+    lens = _block_lens(wl)
+    nb = plan.info.nb
+    f_valid = 0.0
+    for r in range(len(rc)):
+        li = lens[r % nb]
+        f_valid += 4.0 * wl.d * li * sum(lens[j] for j in cols[rp[r]:rp[r + 1]])
+    density = nnz / (len(rc) * nb)
+
+    peak, peak_sus, hbm, peak_kind = _peaks()
+    attn_ms = statistics.mean(per_call["attention"])
+    achieved = f_tile / (attn_ms * 1e-3) / 1e12
+    traffic = _traffic_from_profile(os.path.join(ROOT, "block_sparse_attention_sba_b200", "csrc",
+                                                 "attn_sm100.cu"))
+    value = ws * f_tile / (mean_step * 1e-3) / 1e12
+    ms_calls = {k: round(statistics.mean(vv), 4) for k, vv in per_call.items()}
+    overhead = (ms_calls["reorder"] + ms_calls["build_mask"] + ms_calls["unreorder"]) / ms_calls["attention"]
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
+        n_e2e = max(3, min(args.steps, 10))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            sa(dq, dk, dv, top_p, wl.top_k, o=o, stream=stream)
+            ho.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if pg:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+        e2e = {"value": ws * f_tile / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": ho.numel() * ho.element_size()}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cores, threads = _cpu_cores()
+        f, sec, desc = cpu_oracle_sample(wl, q, k, v, heads=(0,), blocks_per_head=None)
+        cpu = {"value": f / sec / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc + f"; {sec:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": mean_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": _config(wl, {"density": round(density, 4), "nnz_blocks": nnz,
+                                   "sched": "lpt-persistent"}),
+            "ms_per_call": ms_calls,
+            "attention": {"tflops_tile": achieved,
+                          "tflops_valid": f_valid / (attn_ms * 1e-3) / 1e12,
+                          "frac_of_peak": achieved / peak, "peak_kind": peak_kind,
+                          "frac_of_sustained_peak": achieved / peak_sus if peak_sus else None},
+            "overhead_frac": overhead,
+            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128,128>",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_flops_per_launch": f_tile},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 7 * args.steps,
+            "clocks": clocks, "device_status": sba.sba_status_string(status),
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

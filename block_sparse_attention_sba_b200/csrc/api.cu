@@ -1,0 +1,278 @@
+// api.cu -- the C ABI of libsba: argument validation, plan geometry,
+// workspace layout and the launches behind each entry point of sba.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sba {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+KGeom make_kgeom(const sba_plan* p) {
+  const sba_geometry& G = p->g;
+  KGeom k;
+  k.B = G.B;
+  k.H = G.H;
+  k.T = G.T;
+  k.Hh = G.Hh;
+  k.W = G.W;
+  k.d = G.d;
+  k.ct = G.ct;
+  k.ch = G.ch;
+  k.cw = G.cw;
+  k.bs = p->info.bs;
+  k.nT = p->info.nT;
+  k.nH = p->info.nH;
+  k.nW = p->info.nW;
+  k.nb = p->info.nb;
+  k.Npad = p->info.Npad;
+  k.sB = G.sB;
+  k.sH = G.sH;
+  k.sN = G.sN;
+  k.dv_cw = DivMod(G.cw);
+  k.dv_chcw = DivMod(G.ch * G.cw);
+  k.dv_nW = DivMod(k.nW);
+  k.dv_nH = DivMod(k.nH);
+  k.dv_H = DivMod(G.H);
+  k.dv_nb = DivMod(k.nb);
+  return k;
+}
+
+}  // namespace sba
+
+using namespace sba;
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static sba_status fail(sba_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+static sba_status cuda_fail(cudaError_t e, const char* what) {
+  if (g_err[0] == '\0' || e != cudaErrorInvalidValue)
+    snprintf(g_err, sizeof(g_err), "%s: %s", what, cudaGetErrorString(e));
+  return SBA_ERR_CUDA;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+extern "C" {
+
+sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
+  g_err[0] = '\0';
+  if (!geom || !out) return fail(SBA_ERR_INVALID_ARG, "geom and out must be non-NULL");
+  *out = nullptr;
+  const sba_geometry& G = *geom;
+  if (G.B <= 0 || G.H <= 0 || G.T <= 0 || G.Hh <= 0 || G.W <= 0 || G.d <= 0 || G.ct <= 0 ||
+      G.ch <= 0 || G.cw <= 0)
+    return fail(SBA_ERR_INVALID_ARG, "all sizes must be positive");
+  if (G.dtype != SBA_F32 && G.dtype != SBA_BF16)
+    return fail(SBA_ERR_INVALID_ARG, "dtype must be SBA_F32 or SBA_BF16");
+  const int64_t bs = static_cast<int64_t>(G.ct) * G.ch * G.cw;
+  if (bs != 64 && bs != 128)
+    return fail(SBA_ERR_UNSUPPORTED, "block size ct*ch*cw = %lld; supported: 64, 128", (long long)bs);
+  if (G.dtype == SBA_BF16 && G.d != 64 && G.d != 128)
+    return fail(SBA_ERR_UNSUPPORTED, "bf16 head dim %d; supported: 64, 128", G.d);
+  if (G.dtype == SBA_F32 && G.d != 64)
+    return fail(SBA_ERR_UNSUPPORTED, "f32 head dim %d; supported: 64", G.d);
+  const int64_t nT = (G.T + G.ct - 1) / G.ct, nH = (G.Hh + G.ch - 1) / G.ch, nW = (G.W + G.cw - 1) / G.cw;
+  const int64_t nb = nT * nH * nW;
+  const int64_t N = static_cast<int64_t>(G.T) * G.Hh * G.W;
+  if (nb > 1024) return fail(SBA_ERR_CAPACITY, "%lld blocks per head; at most 1024", (long long)nb);
+  if (G.H > 256) return fail(SBA_ERR_CAPACITY, "H = %d; at most 256", G.H);
+  const int64_t BH = static_cast<int64_t>(G.B) * G.H;
+  if (BH > 65535) return fail(SBA_ERR_CAPACITY, "B*H = %lld; at most 65535", (long long)BH);
+  const int64_t R = BH * nb;
+  const int64_t Npad = nb * bs;
+  if (R * nb >= (1ll << 31) || BH * Npad >= (1ll << 31) || N >= (1ll << 31))
+    return fail(SBA_ERR_CAPACITY, "sizes exceed int32 indexing");
+  if (G.sN < G.d || G.sH < 0 || G.sB < 0)
+    return fail(SBA_ERR_INVALID_ARG, "strides must satisfy sN >= d, sH >= 0, sB >= 0");
+  const int esize = G.dtype == SBA_BF16 ? 2 : 4;
+  const int64_t epv = 16 / esize;
+  if (G.sN % epv || G.sH % epv || G.sB % epv)
+    return fail(SBA_ERR_INVALID_ARG, "strides must be multiples of %lld elements (16 bytes)", (long long)epv);
+
+  sba_plan* p = new (std::nothrow) sba_plan();
+  if (!p) return fail(SBA_ERR_CAPACITY, "out of host memory");
+  p->g = G;
+  p->esize = esize;
+  p->info.nT = static_cast<int32_t>(nT);
+  p->info.nH = static_cast<int32_t>(nH);
+  p->info.nW = static_cast<int32_t>(nW);
+  p->info.nb = static_cast<int32_t>(nb);
+  p->info.bs = static_cast<int32_t>(bs);
+  p->info.Npad = static_cast<int32_t>(Npad);
+  p->info.rows = static_cast<int32_t>(R);
+  p->info.words = static_cast<int32_t>((nb + 31) / 32);
+  p->info.max_nnz = R * nb;
+  p->ws_ctrl = 0;
+  p->ws_qbar = 256;
+  const size_t pooled = align256(static_cast<size_t>(R) * G.d * sizeof(float));
+  p->ws_kbar = p->ws_qbar + pooled;
+  p->info.workspace_bytes = p->ws_kbar + pooled;
+  p->wait_budget_ns = 4000000000ull;  // 4 s: no healthy wait comes near it
+  const char* env = getenv("SBA_WAIT_BUDGET_NS");
+  if (env) {
+    unsigned long long v = strtoull(env, nullptr, 10);
+    if (v >= 1000ull && v <= 60000000000ull) p->wait_budget_ns = v;
+  }
+  *out = p;
+  return SBA_OK;
+}
+
+void sba_plan_destroy(sba_plan* plan) { delete plan; }
+
+sba_status sba_plan_query(const sba_plan* plan, sba_plan_info* info) {
+  if (!plan || !info) return fail(SBA_ERR_INVALID_ARG, "plan and info must be non-NULL");
+  *info = plan->info;
+  return SBA_OK;
+}
+
+sba_status sba_workspace_init(const sba_plan* plan, void* workspace, void* stream) {
+  g_err[0] = '\0';
+  if (!plan || !workspace) return fail(SBA_ERR_INVALID_ARG, "plan and workspace must be non-NULL");
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(Ctrl), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "cudaMemsetAsync");
+}
+
+sba_status sba_reorder(const sba_plan* plan, const void* q, const void* k, const void* v, void* qt,
+                       void* kt, void* vt, void* stream) {
+  g_err[0] = '\0';
+  if (!plan) return fail(SBA_ERR_INVALID_ARG, "plan must be non-NULL");
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {qt, kt, vt};
+  for (int i = 0; i < 3; ++i) {
+    if ((src[i] == nullptr) != (dst[i] == nullptr))
+      return fail(SBA_ERR_INVALID_ARG, "tensor %d: source and destination must both be NULL or both set", i);
+    if (src[i] && (!aligned16(src[i]) || !aligned16(dst[i])))
+      return fail(SBA_ERR_INVALID_ARG, "tensor %d: pointers must be 16-byte aligned", i);
+  }
+  cudaError_t e = launch_reorder(plan, 0, src, dst, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_reorder launch");
+}
+
+sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o, void* stream) {
+  g_err[0] = '\0';
+  if (!plan || !ot || !o) return fail(SBA_ERR_INVALID_ARG, "plan, ot and o must be non-NULL");
+  if (!aligned16(ot) || !aligned16(o)) return fail(SBA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const void* src[3] = {ot, nullptr, nullptr};
+  void* dst[3] = {o, nullptr, nullptr};
+  cudaError_t e = launch_reorder(plan, 1, src, dst, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_unreorder launch");
+}
+
+sba_status sba_build_mask(const sba_plan* plan, const void* qt, const void* kt, const float* top_p,
+                          int32_t top_k, uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
+                          int32_t* col_idx, int32_t* work_order, void* workspace, void* stream) {
+  g_err[0] = '\0';
+  if (!plan || !qt || !kt || !top_p || !bitmask || !row_cnt || !row_ptr || !col_idx || !work_order ||
+      !workspace)
+    return fail(SBA_ERR_INVALID_ARG, "sba_build_mask: NULL argument");
+  if (!aligned16(qt) || !aligned16(kt) || !aligned16(workspace))
+    return fail(SBA_ERR_INVALID_ARG, "qt, kt and workspace must be 16-byte aligned");
+  if (top_k < 0) return fail(SBA_ERR_INVALID_ARG, "top_k must be >= 0");
+  for (int h = 0; h < plan->g.H; ++h) {
+    const float p = top_p[h];
+    if (!(p > 0.0f) || !(p <= 1.0f))
+      return fail(SBA_ERR_INVALID_ARG, "top_p[%d] = %g; must lie in (0, 1]", h, (double)p);
+  }
+  cudaError_t e = launch_build_mask(plan, qt, kt, top_p, top_k, bitmask, row_cnt, row_ptr, col_idx,
+                                    work_order, workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_build_mask launch");
+}
+
+sba_status sba_attention(const sba_plan* plan, const void* qt, const void* kt, const void* vt,
+                         const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work_order,
+                         void* ot, float* lse, int32_t sched, uint64_t* trace, void* workspace,
+                         void* stream) {
+  g_err[0] = '\0';
+  if (!plan || !qt || !kt || !vt || !row_ptr || !col_idx || !ot || !workspace)
+    return fail(SBA_ERR_INVALID_ARG, "sba_attention: NULL argument");
+  if (sched != SBA_SCHED_LPT && sched != SBA_SCHED_HEAD_MAJOR)
+    return fail(SBA_ERR_INVALID_ARG, "sched must be SBA_SCHED_LPT or SBA_SCHED_HEAD_MAJOR");
+  if (sched == SBA_SCHED_LPT && !work_order && plan->g.dtype == SBA_BF16)
+    return fail(SBA_ERR_INVALID_ARG, "SBA_SCHED_LPT needs work_order");
+  if (!aligned16(qt) || !aligned16(kt) || !aligned16(vt) || !aligned16(ot))
+    return fail(SBA_ERR_INVALID_ARG, "qt, kt, vt and ot must be 16-byte aligned");
+  cudaError_t e = launch_attention(plan, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse, sched,
+                                   trace, workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_attention launch");
+}
+
+sba_status sba_check_device_status(const sba_plan* plan, void* workspace, void* stream) {
+  g_err[0] = '\0';
+  if (!plan || !workspace) return fail(SBA_ERR_INVALID_ARG, "plan and workspace must be non-NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+  e = cudaMemset(workspace, 0, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+  if (word & kStatusTimeout) return fail(SBA_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up");
+  if (word & kStatusCheck) return fail(SBA_ERR_DEVICE_CHECK, "a device-side input check failed");
+  return SBA_OK;
+}
+
+sba_status sba_debug_timeout_probe(const sba_plan* plan, void* workspace, uint64_t timeout_ns,
+                                   void* stream) {
+  g_err[0] = '\0';
+  if (!plan || !workspace) return fail(SBA_ERR_INVALID_ARG, "plan and workspace must be non-NULL");
+  if (timeout_ns < 1000ull || timeout_ns > 10000000000ull)
+    return fail(SBA_ERR_INVALID_ARG, "timeout_ns must lie in [1e3, 1e10]");
+  cudaError_t e = launch_timeout_probe(workspace, timeout_ns, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "timeout probe launch");
+}
+
+sba_status sba_perm_export(const sba_plan* plan, int32_t* slot_of_token) {
+  if (!plan || !slot_of_token) return fail(SBA_ERR_INVALID_ARG, "plan and output must be non-NULL");
+  const sba_geometry& G = plan->g;
+  const int nH = plan->info.nH, nW = plan->info.nW, bs = plan->info.bs;
+  int64_t n = 0;
+  for (int t = 0; t < G.T; ++t)
+    for (int h = 0; h < G.Hh; ++h)
+      for (int w = 0; w < G.W; ++w, ++n) {
+        const int blk = ((t / G.ct) * nH + h / G.ch) * nW + w / G.cw;
+        const int off = ((t % G.ct) * G.ch + h % G.ch) * G.cw + w % G.cw;
+        slot_of_token[n] = blk * bs + off;
+      }
+  return SBA_OK;
+}
+
+int32_t sba_attention_grid_size(void) { return attention_grid_size(); }
+
+const char* sba_status_string(sba_status s) {
+  switch (s) {
+    case SBA_OK: return "SBA_OK";
+    case SBA_ERR_INVALID_ARG: return "SBA_ERR_INVALID_ARG";
+    case SBA_ERR_UNSUPPORTED: return "SBA_ERR_UNSUPPORTED";
+    case SBA_ERR_CUDA: return "SBA_ERR_CUDA";
+    case SBA_ERR_CAPACITY: return "SBA_ERR_CAPACITY";
+    case SBA_ERR_DEVICE_TIMEOUT: return "SBA_ERR_DEVICE_TIMEOUT";
+    case SBA_ERR_DEVICE_CHECK: return "SBA_ERR_DEVICE_CHECK";
+  }
+  return "SBA_ERR_UNKNOWN";
+}
+
+const char* sba_last_error(void) { return g_err; }
+
+}  // extern "C"

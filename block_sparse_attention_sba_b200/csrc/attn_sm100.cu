@@ -1,0 +1,775 @@
+// attn_sm100.cu -- block-sparse attention forward on B200 tensor cores
+// (FVAttn: Adaptive Sparse Attention with Runtime Load Balancing for Video
+// Generation, abstract: attention over the materialised Top-p / Top-k block
+// mask; uneven per-head workloads absorbed by the scheduler).
+//
+// Work item = one mask row (b, h, query block i): a 128-row query tile and the
+// row's selected key blocks, each a contiguous [bs x d] bf16 tile of the
+// cube-ordered kt / vt. Per item and key block j:
+//   S = Q K_j^T        tcgen05.mma kind::f16, A = Q (smem, K-major),
+//                      B = K_j (smem, K-major), fp32 accumulator in TMEM
+//   P = exp2(S*c - m)  online softmax in fp32 on CUDA cores, one TMEM lane
+//                      (query row) per thread; P rounded to bf16 and written
+//                      back over S in TMEM
+//   O += P V_j         tcgen05.mma with A = P from TMEM, B = V_j (smem,
+//                      MN-major), fp32 accumulator in TMEM
+// Warp roles (192 threads, one CTA per SM):
+//   warps 0-3  softmax + epilogue (thread t owns TMEM lane / query row t)
+//   warp  4    producer: fetches work items, TMA-loads Q and the K/V tiles into
+//              a ring of shared-memory slots in the order the MMAs use them
+//              (K0, K1, V0, K2, V1, ...)
+//   warp  5    MMA issuer (one thread) and TMEM owner
+// Rescaling of O is skipped while the running row max grows by less than
+// 2^8 (the final normalisation uses the same reference max, so the result is
+// exact up to rounding); padding keys of edge cubes are masked to -inf.
+// Scheduler: SBA_SCHED_LPT launches one persistent CTA per SM that takes rows
+// in longest-first work order from an atomic counter (the counter resets
+// itself when the last CTA exits); SBA_SCHED_HEAD_MAJOR launches one CTA per
+// row in (b, h, i) order. Every wait is bounded (status bit + clean exit).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sba {
+
+namespace {
+
+constexpr int kSmemLimit = 232448;  // 227 KB: opt-in shared memory per CTA
+constexpr int kThreads = 192;
+
+template <int D, int BS>
+struct Cfg {
+  static constexpr int M = 128;
+  static constexpr int PANELS = D / 64;  // 128-byte column panels along d
+  static constexpr int Q_BYTES = M * D * 2;
+  static constexpr int TILE_BYTES = BS * D * 2;
+  static constexpr int CTRL_BYTES = 1024;
+  static constexpr int NSLOT_RAW = (kSmemLimit - 1024 - CTRL_BYTES - Q_BYTES) / TILE_BYTES;
+  static constexpr int NSLOT = NSLOT_RAW > 8 ? 8 : NSLOT_RAW;
+  static constexpr int SMEM_USED = 1024 + Q_BYTES + NSLOT * TILE_BYTES + CTRL_BYTES;
+  // Request at least 120 KB so that only one CTA (one 512-column TMEM
+  // allocation) is ever resident per SM.
+  static constexpr int SMEM = SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(M, BS, 0, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(M, D, 0, 1);
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S1 = 128, COL_O = 256;
+  // barrier indices
+  static constexpr int B_QF = 0, B_QE = 1, B_SF = 2, B_SE = B_SF + NSLOT, B_S = B_SE + NSLOT,
+                       B_P = B_S + 2, B_OD = B_P + 2, B_OF = B_OD + 1, B_OE = B_OF + 1,
+                       B_IF = B_OE + 1, B_IE = B_IF + 2, B_DR = B_IE + 2, NBAR = B_DR + 1;
+  static_assert(NSLOT >= 2, "need at least two K/V slots");
+  static_assert(NBAR * 8 <= 256, "barrier area");
+  static_assert(SMEM <= kSmemLimit, "shared memory budget");
+};
+
+struct AttnParams {
+  KGeom g;
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const int32_t* work_order;
+  __nv_bfloat16* ot;
+  float* lse;
+  uint64_t* trace;
+  Ctrl* ctrl;
+  int R;
+  int sched;
+  uint64_t budget_ns;
+  float scale_log2;
+};
+
+// Tile t of an item with n key blocks, in MMA consumption order:
+// K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1).
+__device__ __forceinline__ void tile_of(int t, int n, int& is_v, int& blk) {
+  if (t == 0) {
+    is_v = 0;
+    blk = 0;
+  } else if (t & 1) {
+    const int kb = (t + 1) >> 1;
+    if (kb < n) {
+      is_v = 0;
+      blk = kb;
+    } else {
+      is_v = 1;
+      blk = n - 1;
+    }
+  } else {
+    is_v = 1;
+    blk = (t >> 1) - 1;
+  }
+}
+
+// Wait that ignores the abort flag (used to drain in-flight async work).
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t budget_ns,
+                                                uint32_t* status) {
+  volatile int never = 0;
+  return mbar_wait(bar, parity, budget_ns, &never, status);
+}
+
+__device__ __forceinline__ int block_type(const KGeom& g, int j) {
+  uint32_t rest, tw, tt, th;
+  g.dv_nW.divmod(static_cast<uint32_t>(j), rest, tw);
+  g.dv_nH.divmod(rest, tt, th);
+  return ((static_cast<int>(tt) == g.nT - 1) << 2) | ((static_cast<int>(th) == g.nH - 1) << 1) |
+         (static_cast<int>(tw) == g.nW - 1);
+}
+
+template <int D, int BS>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
+  using C = Cfg<D, BS>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sQ = sm;
+  unsigned char* sSlots = sm + C::Q_BYTES;
+  unsigned char* ctl = sSlots + C::NSLOT * C::TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 260);
+  int* ring = reinterpret_cast<int*>(ctl + 272);        // [2][4]
+  uint32_t* emask = reinterpret_cast<uint32_t*>(ctl + 320);  // [8][4]
+  int* efull = reinterpret_cast<int*>(ctl + 448);            // [8]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const KGeom& g = P.g;
+  uint32_t* status = &P.ctrl->status;
+  const uint64_t budget = P.budget_ns;
+  auto bar = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_QF), 1);
+    mbar_init(bar(C::B_QE), 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(bar(C::B_SF + s), 1);
+      mbar_init(bar(C::B_SE + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::B_S + b), 1);
+      mbar_init(bar(C::B_P + b), 128);
+      mbar_init(bar(C::B_IF + b), 1);
+      mbar_init(bar(C::B_IE + b), 5);
+    }
+    mbar_init(bar(C::B_OD), 1);
+    mbar_init(bar(C::B_OF), 1);
+    mbar_init(bar(C::B_OE), 4);
+    mbar_init(bar(C::B_DR), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x >= 32 && threadIdx.x < 40) {
+    // validity masks of the 8 edge-cube types (bit 2: last in t, 1: in h, 0: in w)
+    const int ty = threadIdx.x - 32;
+    const int vt = (ty & 4) ? g.T - (g.nT - 1) * g.ct : g.ct;
+    const int vh = (ty & 2) ? g.Hh - (g.nH - 1) * g.ch : g.ch;
+    const int vw = (ty & 1) ? g.W - (g.nW - 1) * g.cw : g.cw;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    for (int c = 0; c < BS; ++c) {
+      const int lt = c / (g.ch * g.cw), lh = (c / g.cw) % g.ch, lw = c % g.cw;
+      if (lt < vt && lh < vh && lw < vw) w[c >> 5] |= 1u << (c & 31);
+    }
+    for (int k = 0; k < 4; ++k) emask[ty * 4 + k] = w[k];
+    efull[ty] = (vt == g.ct && vh == g.ch && vw == g.cw) ? 1 : 0;
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+    uint32_t items = 0, tiles = 0, qloads = 0;
+    bool ok = true;
+    while (ok) {
+      int row = -1;
+      if (P.sched == SBA_SCHED_LPT) {
+        int idx = 0;
+        if (lane == 0) idx = static_cast<int>(atomicAdd(&P.ctrl->work_next, 1u));
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        if (idx < P.R) {
+          row = __ldg(&P.work_order[idx]);
+          if (row < 0 || row >= P.R) {
+            if (lane == 0) atomicOr(status, kStatusCheck);
+            row = -1;
+          }
+        }
+      } else {
+        row = (items == 0) ? static_cast<int>(blockIdx.x) : -1;
+      }
+      int start = 0, n = 0;
+      if (row >= 0) {
+        start = __ldg(&P.row_ptr[row]);
+        n = __ldg(&P.row_ptr[row + 1]) - start;
+        if (n < 0 || n > g.nb) {
+          if (lane == 0) atomicOr(status, kStatusCheck);
+          n = n < 0 ? 0 : g.nb;
+        }
+      }
+      const int rs = items & 1;
+      if (items >= 2) {
+        int w = 0;
+        if (lane == 0) w = mbar_wait(bar(C::B_IE + rs), ((items >> 1) - 1) & 1, budget, abort_flag, status);
+        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        if (!ok) break;
+      }
+      if (lane == 0) {
+        ring[rs * 4 + 0] = row;
+        ring[rs * 4 + 1] = n;
+        ring[rs * 4 + 2] = start;
+        mbar_arrive(bar(C::B_IF + rs));
+      }
+      ++items;
+      if (row < 0) break;
+      if (n == 0) continue;
+      uint32_t bh, iq;
+      g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
+      const int rows_base = static_cast<int>(bh) * g.Npad;
+      if (qloads >= 1) {
+        int w = 0;
+        if (lane == 0) w = mbar_wait(bar(C::B_QE), (qloads - 1) & 1, budget, abort_flag, status);
+        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        if (!ok) break;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(C::B_QF), C::Q_BYTES);
+        for (int p = 0; p < C::PANELS; ++p)
+          tma_load_2d(smem_u32(sQ) + p * C::M * 128, &tmQ, p * 64, rows_base + static_cast<int>(iq) * BS,
+                      bar(C::B_QF));
+      }
+      ++qloads;
+      int ck = 0, cv = 0, ckb = -32, cvb = -32;
+      for (int t = 0; t < 2 * n; ++t) {
+        int isv, blk;
+        tile_of(t, n, isv, blk);
+        const int cb = blk & ~31;
+        int j;
+        if (!isv) {
+          if (cb != ckb) {
+            ckb = cb;
+            ck = (cb + lane < n) ? __ldg(&P.col_idx[start + cb + lane]) : 0;
+          }
+          j = __shfl_sync(0xffffffffu, ck, blk & 31);
+        } else {
+          if (cb != cvb) {
+            cvb = cb;
+            cv = (cb + lane < n) ? __ldg(&P.col_idx[start + cb + lane]) : 0;
+          }
+          j = __shfl_sync(0xffffffffu, cv, blk & 31);
+        }
+        if (j < 0 || j >= g.nb) {
+          if (lane == 0) atomicOr(status, kStatusCheck);
+          j = 0;
+        }
+        const int s = static_cast<int>(tiles % C::NSLOT);
+        const uint32_t r = tiles / C::NSLOT;
+        if (r >= 1) {
+          int w = 0;
+          if (lane == 0) w = mbar_wait(bar(C::B_SE + s), (r - 1) & 1, budget, abort_flag, status);
+          ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+          if (!ok) break;
+        }
+        if (lane == 0) {
+          const uint32_t dst = smem_u32(sSlots + s * C::TILE_BYTES);
+          mbar_arrive_expect_tx(bar(C::B_SF + s), C::TILE_BYTES);
+          for (int p = 0; p < C::PANELS; ++p)
+            tma_load_2d(dst + p * BS * 128, isv ? &tmV : &tmK, p * 64, rows_base + j * BS,
+                        bar(C::B_SF + s));
+        }
+        ++tiles;
+      }
+    }
+    if (*abort_flag && lane == 0) {
+      // let every TMA load this CTA issued land before shared memory goes away
+      for (int s = 0; s < C::NSLOT; ++s) {
+        const uint32_t uses = tiles / C::NSLOT + (static_cast<uint32_t>(s) < tiles % C::NSLOT ? 1u : 0u);
+        if (uses) mbar_wait_drain(bar(C::B_SF + s), (uses - 1) & 1, budget, status);
+      }
+      if (qloads) mbar_wait_drain(bar(C::B_QF), (qloads - 1) & 1, budget, status);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t items = 0, tiles = 0, sblocks = 0, qloads = 0, ouses = 0;
+    bool ok = true;
+    auto wait1 = [&](int b, uint32_t parity) -> bool {
+      int w = 0;
+      if (lane == 0) w = mbar_wait(bar(b), parity, budget, abort_flag, status);
+      return __shfl_sync(0xffffffffu, w, 0) != 0;
+    };
+    const uint32_t q_addr = smem_u32(sQ);
+    auto issue_S = [&]() -> bool {
+      const int s = static_cast<int>(tiles % C::NSLOT);
+      if (!wait1(C::B_SF + s, (tiles / C::NSLOT) & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sb = sblocks & 1;
+        const uint32_t dS = tmem + (sb ? C::COL_S1 : 0u);
+        const uint32_t k_addr = smem_u32(sSlots + s * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * (C::M * 128) + off, 16, 1024);
+          const uint64_t b = smem_desc_sw128(k_addr + (kk >> 2) * (BS * 128) + off, 16, 1024);
+          mma_ss(dS, a, b, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_S + sb));
+        mma_commit(bar(C::B_SE + s));
+      }
+      __syncwarp();
+      ++tiles;
+      ++sblocks;
+      return true;
+    };
+    auto issue_PV = [&](uint32_t gblk, bool first) -> bool {
+      const uint32_t sb = gblk & 1;
+      if (!wait1(C::B_P + sb, (gblk >> 1) & 1)) return false;
+      const int s = static_cast<int>(tiles % C::NSLOT);
+      if (!wait1(C::B_SF + s, (tiles / C::NSLOT) & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t aP = tmem + (sb ? C::COL_S1 : 0u);
+        const uint32_t v_addr = smem_u32(sSlots + s * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk) {
+          const uint64_t b = smem_desc_sw128(v_addr + kk * 2048, BS * 128, 1024);
+          mma_ts(tmem + C::COL_O, aP + kk * 8, b, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_OD));
+        mma_commit(bar(C::B_SE + s));
+      }
+      __syncwarp();
+      ++tiles;
+      return true;
+    };
+    while (ok) {
+      const int rs = items & 1;
+      ok = wait1(C::B_IF + rs, (items >> 1) & 1);
+      if (!ok) break;
+      const int row = ring[rs * 4 + 0], n = ring[rs * 4 + 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_IE + rs));
+      ++items;
+      if (row < 0) break;
+      if (n == 0) continue;
+      ok = wait1(C::B_QF, qloads & 1);
+      ++qloads;
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t pbase = sblocks;
+      if (!issue_S()) { ok = false; break; }
+      if (n == 1 && lane == 0) mma_commit(bar(C::B_QE));
+      for (int i = 0; i < n; ++i) {
+        if (i + 1 < n) {
+          if (!issue_S()) { ok = false; break; }
+          if (i + 2 == n && lane == 0) mma_commit(bar(C::B_QE));
+        }
+        if (i == 0 && ouses >= 1) {
+          if (!wait1(C::B_OE, (ouses - 1) & 1)) { ok = false; break; }
+        }
+        if (!issue_PV(pbase + i, i == 0)) { ok = false; break; }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(bar(C::B_OF));
+      __syncwarp();
+      ++ouses;
+    }
+    if (*abort_flag && lane == 0) {
+      mma_commit(bar(C::B_DR));
+      mbar_wait_drain(bar(C::B_DR), 0, budget, status);
+    }
+  } else {
+    // ------------------------------------------------ softmax + epilogue
+    const int t = threadIdx.x;  // query row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = P.scale_log2;
+    uint32_t items = 0, sblocks = 0, pvs = 0, ouses = 0;
+    bool ok = true;
+    while (ok) {
+      const int rs = items & 1;
+      ok = mbar_wait(bar(C::B_IF + rs), (items >> 1) & 1, budget, abort_flag, status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int row = ring[rs * 4 + 0], n = ring[rs * 4 + 1], start = ring[rs * 4 + 2];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_IE + rs));
+      ++items;
+      if (row < 0) break;
+      const uint64_t t_start = globaltimer_ns();
+      uint32_t bh, iq;
+      g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
+      const int qtype = block_type(g, static_cast<int>(iq));
+      const bool qvalid = (t < BS) && ((emask[qtype * 4 + (t >> 5)] >> (t & 31)) & 1u);
+      const int64_t orow = static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(iq) * BS + t;
+      __nv_bfloat16* optr = P.ot + orow * D;
+      if (n == 0) {
+        if (t < BS) {
+          for (int c = 0; c < D; c += 8)
+            *reinterpret_cast<uint4*>(optr + c) = make_uint4(0u, 0u, 0u, 0u);
+          if (P.lse) P.lse[orow] = qvalid ? -INFINITY : 0.f;
+        }
+      } else {
+        float m = -INFINITY, l = 0.f;
+        int jn = __ldg(&P.col_idx[start]);
+        for (int i = 0; i < n; ++i) {
+          const int j = (jn < 0 || jn >= g.nb) ? 0 : jn;
+          if (i + 1 < n) jn = __ldg(&P.col_idx[start + i + 1]);
+          const uint32_t sb = sblocks & 1;
+          ok = mbar_wait(bar(C::B_S + sb), (sblocks >> 1) & 1, budget, abort_flag, status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t scol = tmem + lane_off + (sb ? C::COL_S1 : 0u);
+          uint32_t sr[BS];
+#pragma unroll
+          for (int c = 0; c < BS / 32; ++c)
+            tmem_ld32(scol + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          tmem_ld_wait();
+          float s[BS];
+#pragma unroll
+          for (int e = 0; e < BS; ++e) s[e] = __uint_as_float(sr[e]);
+          const int kt = block_type(g, j);
+          if (!efull[kt]) {
+#pragma unroll
+            for (int c = 0; c < BS / 32; ++c) {
+              const uint32_t w = emask[kt * 4 + c];
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (!((w >> e) & 1u)) s[c * 32 + e] = -INFINITY;
+            }
+          }
+          float mx = s[0];
+#pragma unroll
+          for (int e = 1; e < BS; ++e) mx = fmaxf(mx, s[e]);
+          const float mblk = mx * sl2;
+          float m_new = m, alpha = 1.f;
+          if (i == 0) {
+            m_new = mblk;
+          } else if (mblk > m + 8.0f) {
+            m_new = mblk;
+            alpha = ex2_approx(m - m_new);
+          }
+          if (__any_sync(0xffffffffu, i > 0 && m_new != m)) {
+            // O holds PV up to block i-1: wait for it, then rescale this row
+            ok = mbar_wait(bar(C::B_OD), (pvs + i - 1) & 1, budget, abort_flag, status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32(tmem + lane_off + C::COL_O + c * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st32(tmem + lane_off + C::COL_O + c * 32, r);
+            }
+            tmem_st_wait();
+          }
+          l *= alpha;
+          m = m_new;
+          const float neg_m = -m;
+          float rsum = 0.f;
+#pragma unroll
+          for (int c = 0; c < BS / 64; ++c) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * e], sl2, neg_m));
+              const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * e + 1], sl2, neg_m));
+              rsum += p0 + p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            tmem_st32(scol + c * 32, pk);
+          }
+          tmem_st_wait();
+          l += rsum;
+          tc_fence_before();
+          mbar_arrive(bar(C::B_P + sb));
+          ++sblocks;
+        }
+        if (!ok) break;
+        ok = mbar_wait(bar(C::B_OF), ouses & 1, budget, abort_flag, status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t orr[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          tmem_ld32(tmem + lane_off + C::COL_O + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&orr[c * 32]));
+        tmem_ld_wait();
+        float o[D];
+#pragma unroll
+        for (int e = 0; e < D; ++e) o[e] = __uint_as_float(orr[e]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_OE));
+        ++ouses;
+        pvs += n;
+        if (t < BS) {
+          const float inv = qvalid ? 1.0f / l : 0.f;
+#pragma unroll
+          for (int c = 0; c < D; c += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(o[c + 0] * inv, o[c + 1] * inv);
+            v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
+            v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
+            v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
+            *reinterpret_cast<uint4*>(optr + c) = v;
+          }
+          if (P.lse) P.lse[orow] = qvalid ? (m * 0.69314718055994531f + logf(l)) : 0.f;
+        }
+      }
+      if (P.trace && t == 0) {
+        P.trace[static_cast<int64_t>(row) * 3 + 0] = t_start;
+        P.trace[static_cast<int64_t>(row) * 3 + 1] = globaltimer_ns();
+        P.trace[static_cast<int64_t>(row) * 3 + 2] = smid();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (P.sched == SBA_SCHED_LPT && threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t prev = atomicAdd(&P.ctrl->cta_done, 1u);
+    if (prev == gridDim.x - 1) {
+      atomicExch(&P.ctrl->work_next, 0u);
+      atomicExch(&P.ctrl->cta_done, 0u);
+      __threadfence();
+    }
+  }
+}
+
+// ---------------------------------------------------------------- fp32 path
+// fp32 inputs keep fp32 arithmetic end to end (rounding them to bf16 would
+// cost ~4e-2 max-abs on unit-scale data): one CTA per row, one thread per
+// query slot, K/V tiles staged in shared memory, exact fp32 online softmax.
+template <int D>
+__global__ void __launch_bounds__(128)
+    attn_f32_kernel(KGeom g, const float* __restrict__ qt, const float* __restrict__ kt,
+                    const float* __restrict__ vt, const int32_t* __restrict__ row_ptr,
+                    const int32_t* __restrict__ col_idx, float* __restrict__ ot,
+                    float* __restrict__ lse, uint64_t* __restrict__ trace, uint32_t* status,
+                    float scale_log2) {
+  extern __shared__ float fsm[];
+  const int BS = g.bs;
+  float* Ks = fsm;                  // [BS][D+1]
+  float* Vs = fsm + BS * (D + 1);   // [BS][D]
+  const int row = blockIdx.x;
+  const int t = threadIdx.x;
+  const uint64_t t_start = globaltimer_ns();
+  uint32_t bh, iq;
+  g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
+  const int64_t head = static_cast<int64_t>(bh) * g.Npad;
+
+  auto valid_slot = [&](int blk, int c) -> bool {
+    uint32_t rest, tw, tt, th;
+    g.dv_nW.divmod(static_cast<uint32_t>(blk), rest, tw);
+    g.dv_nH.divmod(rest, tt, th);
+    uint32_t lt, r2, lh, lw;
+    g.dv_chcw.divmod(static_cast<uint32_t>(c), lt, r2);
+    g.dv_cw.divmod(r2, lh, lw);
+    return (static_cast<int>(tt * g.ct + lt) < g.T) && (static_cast<int>(th * g.ch + lh) < g.Hh) &&
+           (static_cast<int>(tw * g.cw + lw) < g.W);
+  };
+  const bool active = t < BS;
+  const bool qvalid = active && valid_slot(static_cast<int>(iq), t);
+  const int64_t qrow = head + static_cast<int64_t>(iq) * BS + t;
+  float q[D], o[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    q[c] = active ? qt[qrow * D + c] * scale_log2 : 0.f;
+    o[c] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  const int start = row_ptr[row];
+  int n = row_ptr[row + 1] - start;
+  if (n < 0 || n > g.nb) {
+    if (t == 0) atomicOr(status, kStatusCheck);
+    n = n < 0 ? 0 : g.nb;
+  }
+  for (int i = 0; i < n; ++i) {
+    int j = col_idx[start + i];
+    if (j < 0 || j >= g.nb) {
+      if (t == 0) atomicOr(status, kStatusCheck);
+      j = 0;
+    }
+    __syncthreads();
+    for (int e = t; e < BS * D; e += blockDim.x) {
+      const int r = e / D, c = e % D;
+      const int64_t src = (head + static_cast<int64_t>(j) * BS + r) * D + c;
+      Ks[r * (D + 1) + c] = kt[src];
+      Vs[r * D + c] = vt[src];
+    }
+    __syncthreads();
+    if (!active) continue;
+    for (int c = 0; c < BS; ++c) {
+      if (!valid_slot(j, c)) continue;
+      float s = 0.f;
+#pragma unroll
+      for (int x = 0; x < D; ++x) s = fmaf(q[x], Ks[c * (D + 1) + x], s);
+      if (s > m) {
+        const float a = exp2f(m - s);
+        l *= a;
+#pragma unroll
+        for (int x = 0; x < D; ++x) o[x] *= a;
+        m = s;
+      }
+      const float p = exp2f(s - m);
+      l += p;
+#pragma unroll
+      for (int x = 0; x < D; ++x) o[x] = fmaf(p, Vs[c * D + x], o[x]);
+    }
+  }
+  if (active) {
+    const float inv = (qvalid && n > 0) ? 1.0f / l : 0.f;
+#pragma unroll
+    for (int c = 0; c < D; ++c) ot[qrow * D + c] = o[c] * inv;
+    if (lse) lse[qrow] = !qvalid ? 0.f : (n > 0 ? m * 0.69314718055994531f + logf(l) : -INFINITY);
+  }
+  if (trace && t == 0) {
+    trace[static_cast<int64_t>(row) * 3 + 0] = t_start;
+    trace[static_cast<int64_t>(row) * 3 + 1] = globaltimer_ns();
+    trace[static_cast<int64_t>(row) * 3 + 2] = smid();
+  }
+}
+
+__global__ void timeout_probe_kernel(Ctrl* ctrl, uint64_t budget_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on this barrier: the bounded wait must give up.
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, budget_ns, &abort_flag, &ctrl->status);
+}
+
+// ----------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int g_grid_size = 0;
+
+template <int D, int BS>
+cudaError_t launch_tc(const sba_plan* p, const void* qt, const void* kt, const void* vt,
+                      const AttnParams& ap, cudaStream_t st) {
+  using C = Cfg<D, BS>;
+  const int64_t rows = static_cast<int64_t>(p->g.B) * p->g.H * p->info.Npad;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, qt, rows, D, 128) || !make_map(&mk, kt, rows, D, BS) ||
+      !make_map(&mv, vt, rows, D, BS)) {
+    set_error("cuTensorMapEncodeTiled unavailable or rejected the tensor");
+    return cudaErrorInvalidValue;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int optin = 0, sms = 0;
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (optin < C::SMEM) {
+    set_error("device offers %d bytes of shared memory per CTA, kernel needs %d", optin, C::SMEM);
+    return cudaErrorInvalidConfiguration;
+  }
+  e = cudaFuncSetAttribute(attn_tc_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int grid = ap.sched == SBA_SCHED_LPT ? std::min(sms, ap.R) : ap.R;
+  if (ap.sched == SBA_SCHED_LPT) g_grid_size = grid;
+  attn_tc_kernel<D, BS><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, ap);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attention_grid_size() { return g_grid_size; }
+
+cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, const void* vt,
+                             const int32_t* row_ptr, const int32_t* col_idx,
+                             const int32_t* work_order, void* ot, float* lse, int sched,
+                             uint64_t* trace, void* workspace, cudaStream_t st) {
+  KGeom g = make_kgeom(p);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(static_cast<char*>(workspace) + p->ws_ctrl);
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(g.d)));
+  if (p->g.dtype == SBA_F32) {
+    const size_t smem = static_cast<size_t>(g.bs) * (2 * g.d + 1) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attn_f32_kernel<64><<<p->info.rows, 128, smem, st>>>(
+        g, static_cast<const float*>(qt), static_cast<const float*>(kt), static_cast<const float*>(vt),
+        row_ptr, col_idx, static_cast<float*>(ot), lse, trace, &ctrl->status, scale_log2);
+    return cudaGetLastError();
+  }
+  AttnParams ap;
+  ap.g = g;
+  ap.row_ptr = row_ptr;
+  ap.col_idx = col_idx;
+  ap.work_order = work_order;
+  ap.ot = static_cast<__nv_bfloat16*>(ot);
+  ap.lse = lse;
+  ap.trace = trace;
+  ap.ctrl = ctrl;
+  ap.R = p->info.rows;
+  ap.sched = sched;
+  ap.budget_ns = p->wait_budget_ns;
+  ap.scale_log2 = scale_log2;
+  if (g.d == 128 && g.bs == 128) return launch_tc<128, 128>(p, qt, kt, vt, ap, st);
+  if (g.d == 128 && g.bs == 64) return launch_tc<128, 64>(p, qt, kt, vt, ap, st);
+  if (g.d == 64 && g.bs == 128) return launch_tc<64, 128>(p, qt, kt, vt, ap, st);
+  if (g.d == 64 && g.bs == 64) return launch_tc<64, 64>(p, qt, kt, vt, ap, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_timeout_probe(void* workspace, uint64_t timeout_ns, cudaStream_t st) {
+  timeout_probe_kernel<<<1, 32, 0, st>>>(static_cast<Ctrl*>(workspace), timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace sba

@@ -1,0 +1,79 @@
+// internal.h -- the plan and the launchers shared by the library's sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sba.h"
+
+struct sba_plan {
+  sba_geometry g;
+  sba_plan_info info;
+  int esize;               // bytes per element (2 or 4)
+  size_t ws_ctrl;          // offset of the control block (status, counters)
+  size_t ws_qbar, ws_kbar; // offsets of the pooled means (fp32 [B*H][nb][d])
+  uint64_t wait_budget_ns; // bounded-wait limit for device waits
+};
+
+namespace sba {
+
+// Control block at the start of every workspace (256 bytes, zero at rest).
+struct Ctrl {
+  uint32_t status;        // kStatusTimeout | kStatusCheck bits
+  uint32_t work_next;     // persistent scheduler: next work_order index
+  uint32_t cta_done;      // persistent scheduler: CTAs that finished
+  uint32_t pad[61];
+};
+static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
+
+// Fast unsigned division by a runtime constant (multiply-high + shift),
+// valid for dividends below 2^31.
+struct DivMod {
+  uint32_t d, mul, shr;
+  __host__ __device__ DivMod() : d(1), mul(0), shr(0) {}
+  __host__ explicit DivMod(uint32_t div) : d(div) {
+    shr = 0;
+    while ((1u << shr) < div) ++shr;
+    // mul = ceil(2^(32+shr) / d) - 2^32 fits in 32 bits for d >= 1
+    uint64_t m = ((1ull << (32 + shr)) + div - 1) / div;
+    mul = static_cast<uint32_t>(m - (1ull << 32));
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    uint32_t t = __umulhi(n, mul);
+    return (t + n) >> shr;  // (t + n) < 2^32 for n < 2^31
+  }
+  __device__ __forceinline__ void divmod(uint32_t n, uint32_t& q, uint32_t& r) const {
+    q = div(n);
+    r = n - q * d;
+  }
+};
+
+// Geometry in the form the kernels take by value.
+struct KGeom {
+  int32_t B, H, T, Hh, W, d, ct, ch, cw, bs, nT, nH, nW, nb, Npad;
+  int64_t sB, sH, sN;
+  DivMod dv_cw, dv_chcw, dv_nW, dv_nH, dv_H, dv_nb;
+};
+
+KGeom make_kgeom(const sba_plan* p);
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_reorder(const sba_plan* p, int direction, const void* src[3], void* dst[3],
+                           cudaStream_t st);
+cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
+                              const float* top_p, int top_k, uint32_t* bitmask, int32_t* row_cnt,
+                              int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
+                              void* workspace, cudaStream_t st);
+cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, const void* vt,
+                             const int32_t* row_ptr, const int32_t* col_idx,
+                             const int32_t* work_order, void* ot, float* lse, int sched,
+                             uint64_t* trace, void* workspace, cudaStream_t st);
+cudaError_t launch_timeout_probe(void* workspace, uint64_t timeout_ns, cudaStream_t st);
+
+// Set by launch_attention when it fails before a launch for a reason that is
+// not a CUDA error (e.g. the tensor-map encoder is unavailable).
+void set_error(const char* fmt, ...);
+
+int attention_grid_size();
+
+}  // namespace sba

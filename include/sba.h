@@ -1,0 +1,204 @@
+/*
+ * sba.h -- C ABI of libsba, training-free Top-p block-sparse self-attention
+ * for video diffusion transformers, built for NVIDIA B200 (sm_100a).
+ *
+ * The method (FVAttn: Adaptive Sparse Attention with Runtime Load Balancing
+ * for Video Generation, abstract): a sparse-routing front end made of
+ * "video-aware block organization", "Top-p routing" and "a Top-k safety
+ * floor" materialises a block mask, and attention then runs over the selected
+ * blocks only; adaptive Top-p gives uneven per-head work, which a scheduler
+ * has to absorb. The four calls below are the four steps of that path:
+ *
+ *   sba_reorder     raster (t,h,w) tokens -> spatio-temporal cube blocks
+ *   sba_build_mask  pooled block scores -> Top-p / Top-k mask (bitmask + CSR)
+ *                   and a longest-first work order
+ *   sba_attention   online-softmax attention over the selected key blocks
+ *   sba_unreorder   cube blocks -> raster tokens
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Geometry: a latent grid of T x Hh x W tokens (N = T*Hh*W), cut into cubes
+ *   of ct x ch x cw tokens; every cube is one block of bs = ct*ch*cw slots.
+ *   The cube grid is nT x nH x nW with nT = ceil(T/ct) etc., nb = nT*nH*nW
+ *   blocks per head and Npad = nb*bs slots per head. A grid that does not
+ *   divide into whole cubes is padded: padding slots keep their geometric
+ *   place inside their cube, hold zeros after sba_reorder, are never attended
+ *   to as keys and produce zero output rows.
+ * - Token order: raster token n = (t*Hh + h)*W + w. Slot of a token:
+ *   blk*bs + ((t%ct)*ch + h%ch)*cw + w%cw with
+ *   blk = ((t/ct)*nH + h/ch)*nW + w/cw (cubes row-major over the cube grid,
+ *   tokens row-major inside a cube).
+ * - Tensors: raster q, k, v, o are [B][H][N][d] with element strides sB, sH,
+ *   sN given in the geometry and d contiguous (so [B][N][H][d] storage is
+ *   accepted). Reordered qt, kt, vt, ot are packed [B][H][Npad][d].
+ * - Rows of the mask: r = (b*H + h)*nb + i for query block i; R = B*H*nb.
+ * - Memory: every buffer is allocated and owned by the caller; the library
+ *   never allocates device memory and never synchronises, except
+ *   sba_check_device_status. Device pointers must be 16-byte aligned.
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *   default stream). Every call is asynchronous on it.
+ * - Errors: arguments are validated on the host before any launch and a
+ *   negative status is returned with a message in sba_last_error(). A failed
+ *   launch returns SBA_ERR_CUDA. Checks that only the device can make (a
+ *   column index out of range, a bounded wait that gave up) set bits in a
+ *   status word inside the workspace; sba_check_device_status reads them.
+ */
+#ifndef SBA_H_
+#define SBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SBA_API __attribute__((visibility("default")))
+#else
+#define SBA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SBA_OK = 0,
+  SBA_ERR_INVALID_ARG = -1,     /* bad pointer, size, stride or value */
+  SBA_ERR_UNSUPPORTED = -2,     /* valid but not built (e.g. an untuned d) */
+  SBA_ERR_CUDA = -3,            /* a CUDA runtime/driver call failed */
+  SBA_ERR_CAPACITY = -4,        /* a size exceeds an int32 index or a limit */
+  SBA_ERR_DEVICE_TIMEOUT = -5,  /* a bounded device-side wait gave up */
+  SBA_ERR_DEVICE_CHECK = -6     /* a device-side input check failed */
+} sba_status;
+
+typedef enum { SBA_F32 = 0, SBA_BF16 = 1 } sba_dtype;
+
+typedef enum {
+  SBA_SCHED_LPT = 0,        /* persistent CTAs, rows taken longest first */
+  SBA_SCHED_HEAD_MAJOR = 1  /* one CTA per row, rows in (b, h, i) order */
+} sba_sched;
+
+/* Geometry of one attention layer (see the conventions above). */
+typedef struct {
+  int32_t B, H;          /* batch, heads */
+  int32_t T, Hh, W;      /* latent grid: frames, height, width */
+  int32_t d;             /* head dimension */
+  int32_t ct, ch, cw;    /* cube extents; bs = ct*ch*cw */
+  int32_t dtype;         /* sba_dtype of q, k, v, o and their reordered forms */
+  int64_t sB, sH, sN;    /* element strides of raster q/k/v/o; d is contiguous */
+} sba_geometry;
+
+/* Sizes derived from a geometry. */
+typedef struct {
+  int32_t nT, nH, nW;        /* cube grid */
+  int32_t nb;                /* blocks per head (query and key) */
+  int32_t bs;                /* slots per block */
+  int32_t Npad;              /* slots per head = nb*bs */
+  int32_t rows;              /* R = B*H*nb mask rows */
+  int32_t words;             /* uint32 words per bitmask row = ceil(nb/32) */
+  int64_t max_nnz;           /* worst-case length of col_idx = R*nb */
+  size_t workspace_bytes;    /* size of the workspace every call below takes */
+} sba_plan_info;
+
+typedef struct sba_plan sba_plan;
+
+/* Validate a geometry and build a host-side plan (no device memory, no CUDA
+ * call). Supported: bs in {64, 128}; bf16 with d in {64, 128}; f32 with d = 64;
+ * nb <= 1024; B*H <= 65535; H <= 256; R*nb < 2^31; strides multiples of 8
+ * elements. Returns SBA_ERR_INVALID_ARG / SBA_ERR_UNSUPPORTED /
+ * SBA_ERR_CAPACITY otherwise. The plan is immutable and may be shared by
+ * threads. */
+SBA_API sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out);
+SBA_API void sba_plan_destroy(sba_plan* plan);
+SBA_API sba_status sba_plan_query(const sba_plan* plan, sba_plan_info* info);
+
+/* Zero the control words at the start of a workspace (status word and the
+ * scheduler's counters). Call once after allocating a workspace, before its
+ * first use; a workspace allocated zero-filled needs no call. */
+SBA_API sba_status sba_workspace_init(const sba_plan* plan, void* workspace, void* stream);
+
+/* Video-aware block organization (FVAttn abstract): gather raster q, k, v into
+ * cube order. Each of the three (src, dst) pairs may be (NULL, NULL) to skip
+ * that tensor. Padding slots are written as zeros. Bit copy: no rounding. */
+SBA_API sba_status sba_reorder(const sba_plan* plan,
+                       const void* q, const void* k, const void* v,
+                       void* qt, void* kt, void* vt, void* stream);
+
+/* Inverse of sba_reorder for the output: ot [B][H][Npad][d] -> o, raster with
+ * the geometry's strides. Padding slots are dropped. Bit copy. */
+SBA_API sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o, void* stream);
+
+/* Block scoring and routing (FVAttn abstract: Top-p routing, Top-k safety
+ * floor). For every row r = (b, h, i):
+ *   Qbar_i, Kbar_j = means of qt, kt over the real tokens of block i, j (fp32)
+ *   P_ij = softmax_j(Qbar_i . Kbar_j / sqrt(d))
+ *   sort j by P_ij descending (ties: lower j first); n_p = the shortest
+ *   prefix whose cumulative mass reaches top_p[h] (all nb when it never does
+ *   or top_p[h] >= 1); keep n = min(nb, max(top_k, n_p)) blocks.
+ * Outputs (device, caller-owned):
+ *   bitmask   uint32 [R][words]; bit j%32 of word j/32 set when block j kept
+ *   row_cnt   int32 [R]; n of every row
+ *   row_ptr   int32 [R+1]; exclusive prefix sum of row_cnt
+ *   col_idx   int32 [>= row_ptr[R]]; kept j of each row, ascending (size it
+ *             for max_nnz, or for a bound the caller knows)
+ *   work_order int32 [R]; rows by row_cnt descending, equal counts by row
+ *             ascending (longest-processing-time-first order)
+ * top_p is a host array [H]; values in (0, 1] are meaningful, p >= 1 keeps
+ * every block. top_k >= 0. Scores are fp32; rows whose cumulative mass at the
+ * cut lies within ~1e-5 of p may differ from an fp64 evaluation. */
+SBA_API sba_status sba_build_mask(const sba_plan* plan, const void* qt, const void* kt,
+                          const float* top_p, int32_t top_k,
+                          uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
+                          int32_t* col_idx, int32_t* work_order,
+                          void* workspace, void* stream);
+
+/* Block-sparse attention forward (FVAttn abstract: attention over the
+ * materialised mask). For every real query slot q of block i:
+ *   o_q = sum_{j in cols(i)} sum_{real keys k of j} softmax(q.k / sqrt(d)) v_k
+ * with the softmax taken over exactly those keys; lse_q = log of its
+ * denominator (natural log, scores already divided by sqrt(d)). bf16 inputs
+ * run on tcgen05 tensor cores (bf16 operands, fp32 accumulation in tensor
+ * memory, fp32 online softmax) and write bf16 ot; f32 inputs run in fp32 on
+ * CUDA cores and write f32 ot. Padding query slots get o = 0 and lse = 0; a
+ * row with no columns gets o = 0 and lse = -inf.
+ *   row_ptr, col_idx  the CSR from sba_build_mask (or any CSR over [0, nb)
+ *                     with at most nb columns per row)
+ *   work_order        int32 [R], required for SBA_SCHED_LPT, ignored (may be
+ *                     NULL) for SBA_SCHED_HEAD_MAJOR
+ *   lse               float [B][H][Npad] or NULL
+ *   trace             NULL, or uint64 [R][3] receiving, per row, the
+ *                     %globaltimer ns at which its CTA started and finished it
+ *                     and the SM id (for the SM idle / tail measurement)
+ * A column index outside [0, nb) is replaced by 0 and flags
+ * SBA_ERR_DEVICE_CHECK in the workspace status word. */
+SBA_API sba_status sba_attention(const sba_plan* plan, const void* qt, const void* kt, const void* vt,
+                         const int32_t* row_ptr, const int32_t* col_idx,
+                         const int32_t* work_order, void* ot, float* lse,
+                         int32_t sched, uint64_t* trace, void* workspace, void* stream);
+
+/* Synchronise `stream`, read and clear the workspace status word. Returns
+ * SBA_OK, SBA_ERR_DEVICE_TIMEOUT or SBA_ERR_DEVICE_CHECK (timeouts win). */
+SBA_API sba_status sba_check_device_status(const sba_plan* plan, void* workspace, void* stream);
+
+/* Failure-detection probe: launch one CTA that waits, with the library's
+ * bounded wait, on a barrier that nothing arrives at, for at most
+ * timeout_ns nanoseconds (1e3..1e10). The wait gives up, flags
+ * SBA_ERR_DEVICE_TIMEOUT in the status word and the kernel returns normally,
+ * leaving the context usable. Used to test the timeout path without a hang. */
+SBA_API sba_status sba_debug_timeout_probe(const sba_plan* plan, void* workspace,
+                                   uint64_t timeout_ns, void* stream);
+
+/* Host-only: write the slot of every raster token, int32 [N]. */
+SBA_API sba_status sba_perm_export(const sba_plan* plan, int32_t* slot_of_token);
+
+/* Number of SMs the persistent attention grid uses on the current device
+ * (0 before the first sba_attention call in this process). */
+SBA_API int32_t sba_attention_grid_size(void);
+
+SBA_API const char* sba_status_string(sba_status status);
+/* Message of the last failed call on this thread ("" if none). */
+SBA_API const char* sba_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBA_H_ */

@@ -1,0 +1,133 @@
+"""The C-ABI library loads on a CPU-only host, exports every symbol that
+include/sba.h declares, validates arguments on the host, and its host-side
+geometry agrees with the oracle. No device call is made here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sba():
+    import block_sparse_attention_sba_b200 as m
+    return m
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sba.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sba_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = _declared_symbols()
+    for s in ["sba_reorder", "sba_build_mask", "sba_attention", "sba_unreorder",
+              "sba_plan_create", "sba_check_device_status", "sba_status_string"]:
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(sba):
+    lib = ctypes.CDLL(sba.LIB_PATH)
+    for s in _declared_symbols():
+        assert hasattr(lib, s), f"{s} declared in sba.h but not exported"
+    assert set(_declared_symbols()) == set(sba.EXPORTED)
+
+
+def test_status_strings(sba):
+    for code in range(-6, 1):
+        assert sba.sba_status_string(code).startswith("SBA_")
+
+
+GEOMS = [
+    (1, 2, 4, 8, 8, 64, (4, 4, 4), "f32"),
+    (1, 8, 8, 16, 16, 64, (4, 4, 4), "bf16"),
+    (1, 40, 21, 30, 52, 128, (2, 8, 8), "bf16"),
+    (1, 24, 33, 45, 80, 128, (2, 8, 8), "bf16"),
+    (2, 3, 5, 9, 7, 64, (2, 4, 8), "bf16"),
+]
+
+
+@pytest.mark.parametrize("B,H,T,Hh,W,d,cube,dt", GEOMS)
+def test_plan_geometry_matches_oracle(sba, B, H, T, Hh, W, d, cube, dt):
+    plan = sba.Plan(B, H, T, Hh, W, d, cube, dt)
+    g = oracle.Geom(T, Hh, W, *cube)
+    inf = plan.info
+    assert (inf.nT, inf.nH, inf.nW, inf.nb, inf.bs, inf.Npad) == (g.nT, g.nH, g.nW, g.nb, g.bs, g.Npad)
+    assert inf.rows == B * H * g.nb and inf.words == (g.nb + 31) // 32
+    assert inf.max_nnz == inf.rows * g.nb
+    assert inf.workspace_bytes >= 256 + 2 * inf.rows * d * 4
+
+
+@pytest.mark.parametrize("T,Hh,W,cube", [(4, 8, 8, (4, 4, 4)), (5, 9, 7, (2, 4, 8)),
+                                         (21, 30, 52, (2, 8, 8)), (3, 3, 3, (1, 8, 8))])
+def test_host_permutation_matches_oracle(sba, T, Hh, W, cube):
+    plan = sba.Plan(1, 1, T, Hh, W, 64, cube, "bf16")
+    got = np.array(sba.sba_perm_export(plan.handle, T * Hh * W))
+    assert np.array_equal(got, oracle.slot_of_token(oracle.Geom(T, Hh, W, *cube)))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), -2),                       # untuned head dim
+    (dict(cube=(2, 4, 4)), -2),             # block of 32
+    (dict(dt="f32", d=128), -2),
+    (dict(T=0), -1),
+    (dict(H=300), -4),
+    (dict(T=200, Hh=64, W=64), -4),         # too many blocks per head
+])
+def test_plan_rejects_bad_geometry(sba, kw, code):
+    args = dict(B=1, H=2, T=4, Hh=8, W=8, d=64, cube=(4, 4, 4), dt="bf16")
+    args.update(kw)
+    with pytest.raises(sba.SbaError) as e:
+        sba.Plan(args["B"], args["H"], args["T"], args["Hh"], args["W"], args["d"], args["cube"],
+                 args["dt"])
+    assert e.value.status == code
+
+
+def test_plan_rejects_unaligned_strides(sba):
+    with pytest.raises(sba.SbaError) as e:
+        sba.Plan(1, 2, 4, 8, 8, 64, (4, 4, 4), "bf16", strides=(4 * 8 * 8 * 64 * 2, 4 * 8 * 8 * 64, 68))
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+
+
+def test_calls_validate_before_any_launch(sba):
+    plan = sba.Plan(1, 2, 4, 8, 8, 64, (4, 4, 4), "bf16")
+    h = plan.handle
+    fake = 1 << 20  # never dereferenced: validation fails first
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_reorder(h, fake, None, None, None, None, None, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_reorder(h, fake + 8, None, None, fake, None, None, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG     # misaligned
+    for bad_p in ([0.0, 0.5], [0.5, 1.5], [float("nan"), 0.5]):
+        with pytest.raises(sba.SbaError) as e:
+            sba.sba_build_mask(h, fake, fake, bad_p, 1, fake, fake, fake, fake, fake, fake, stream=0)
+        assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_build_mask(h, fake, fake, [0.5, 0.5], -1, fake, fake, fake, fake, fake, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_attention(h, fake, fake, fake, fake, fake, fake, fake, None, 7, None, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_attention(h, fake, fake, fake, fake, fake, None, fake, None, sba.SBA_SCHED_LPT,
+                          None, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_debug_timeout_probe(h, fake, 10, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    assert "must" in sba.sba_last_error()
+
+
+def test_binding_has_no_fallback_path():
+    """The package is the C ABI plus marshalling: it must not import the
+    oracle or any compute library."""
+    src = open(os.path.join(ROOT, "block_sparse_attention_sba_b200", "__init__.py")).read()
+    assert "oracle" not in src.replace("no fallback", "")
+    assert "numpy" not in src and "scaled_dot_product" not in src
