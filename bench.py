@@ -46,6 +46,10 @@ def _args():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sched-report", action="store_true")
+    ap.add_argument("--gen-device", choices=["gpu", "cpu"], default="gpu",
+                    help="where the synthetic inputs are generated (cpu: no GPU launches "
+                         "before the timed kernels, for profiler captures)")
     return ap.parse_args()
 
 
@@ -229,6 +233,52 @@ def run_reference(args):
     return 0
 
 
+def sched_report(dev, name="stress", reps=3):
+    """SM idle / tail fraction of sba_attention on the heterogeneous-load
+    workload, persistent longest-first vs one CTA per row in head-major order,
+    from per-row %globaltimer stamps: idle = 1 - sum(row busy time) /
+    (SMs x makespan). Also the per-head spread of selected blocks."""
+    import torch
+
+    import block_sparse_attention_sba_b200 as sba
+    import datagen
+    wl = datagen.WORKLOADS[name]
+    q, k, v = datagen.generate(wl, seed=0, device=dev)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    sa = sba.SparseAttention(plan, device=dev)
+    h = plan.handle
+    sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt)
+    sba.sba_build_mask(h, sa.qt, sa.kt, wl.top_p_per_head(), wl.top_k, sa.bitmask, sa.row_cnt,
+                       sa.row_ptr, sa.col_idx, sa.work_order, sa.workspace)
+    R = plan.info.rows
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    trace = torch.zeros(R * 3, dtype=torch.int64, device=dev)
+    out = {"workload": name}
+    for label, mode in (("lpt_persistent", sba.SBA_SCHED_LPT), ("head_major_grid", sba.SBA_SCHED_HEAD_MAJOR)):
+        best = None
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sba.sba_attention(h, sa.qt, sa.kt, sa.vt, sa.row_ptr, sa.col_idx, sa.work_order, sa.ot,
+                              sa.lse, mode, trace, sa.workspace)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            tr = trace.view(R, 3).cpu()
+            t0 = int(tr[:, 0].min())
+            t1 = int(tr[:, 1].max())
+            busy = float((tr[:, 1] - tr[:, 0]).sum())
+            span = float(t1 - t0)
+            res = {"ms": e0.elapsed_time(e1), "idle_frac": 1.0 - busy / (nsm * span),
+                   "makespan_ms": span * 1e-6, "sms_used": int(torch.unique(tr[:, 2]).numel())}
+            if best is None or res["ms"] < best["ms"]:
+                best = res
+        out[label] = best
+    cnt = sa.row_cnt.view(wl.B * wl.H, plan.info.nb).sum(dim=1).float()
+    out["per_head_blocks_max_over_min"] = float(cnt.max() / cnt.min())
+    out["density"] = float(sa.row_cnt.sum()) / (R * plan.info.nb)
+    return out
+
+
 def run_ours(args):
     import torch
 
@@ -249,7 +299,8 @@ def run_ours(args):
                                 device_id=dev)
         pg = dist
     wl = datagen.WORKLOADS[args.workload]
-    q, k, v = datagen.generate(wl, seed=0, device=dev)
+    gen_dev = dev if args.gen_device == "gpu" else "cpu"
+    q, k, v = datagen.generate(wl, seed=0, device=gen_dev, out_device=dev)
     plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
     sa = sba.SparseAttention(plan, device=dev)
     h = plan.handle
@@ -372,6 +423,10 @@ def run_ours(args):
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": ho.numel() * ho.element_size()}
 
+    sched = None
+    if not args.no_sched_report:
+        sched = sched_report(dev)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cores, threads = _cpu_cores()
@@ -396,6 +451,7 @@ def run_ours(args):
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": f_tile},
+            "scheduler": sched,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 7 * args.steps,
             "clocks": clocks, "device_status": sba.sba_status_string(status),
         }

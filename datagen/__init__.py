@@ -83,6 +83,10 @@ WORKLOADS = {
                         rope_split=(44, 42, 42)),
     "stress": Workload("stress", 1, 40, 21, 30, 52, 128, (2, 8, 8), "bf16", STRESS_P, 8,
                        rope_split=(44, 42, 42), amp_range=(0.2, 3.0)),
+    # the Wan layer cut to 8 heads: same kernels and tile shapes, 0.24 GB of
+    # reordered q/k/v (still larger than L2), used for profiler captures
+    "wan8": Workload("wan8", 1, 8, 21, 30, 52, 128, (2, 8, 8), "bf16", (0.9,), 8,
+                     rope_split=(44, 42, 42)),
 }
 
 
@@ -180,9 +184,9 @@ def generate(wl: Workload, seed: int = 0, device: str | torch.device = "cpu",
             if wl.rope_split is not None:
                 Q = _rope(Q, coords_t, wl.rope_split)
                 K = _rope(K, coords_t, wl.rope_split)
-            q[b, h] = Q.to(out_device).to(dt)
-            k[b, h] = K.to(out_device).to(dt)
-            v[b, h] = torch.from_numpy(vv).to(dt).to(out_device)
+            q[b, h] = Q.to(dt).to(out_device)
+            k[b, h] = K.to(dt).to(out_device)
+            v[b, h] = torch.from_numpy(vv).to(device).to(dt).to(out_device)
     return q, k, v
 
 
