@@ -38,7 +38,8 @@ SBA_SCHED_HEAD_MAJOR = 1
 EXPORTED = ["sba_plan_create", "sba_plan_destroy", "sba_plan_query", "sba_workspace_init",
             "sba_reorder", "sba_unreorder", "sba_build_mask", "sba_attention",
             "sba_check_device_status", "sba_debug_timeout_probe", "sba_perm_export",
-            "sba_attention_grid_size", "sba_status_string", "sba_last_error"]
+            "sba_attention_grid_size", "sba_status_string", "sba_last_error",
+            "sba_build_mask_noalloc"]
 
 
 class sba_geometry(ctypes.Structure):
@@ -68,6 +69,8 @@ _sig = {
     "sba_build_mask": [_vp, _vp, _vp, ctypes.POINTER(ctypes.c_float), _i32, _vp, _vp, _vp, _vp,
                        _vp, _vp, _vp],
     "sba_attention": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp],
+    "sba_build_mask_noalloc": [_vp, _vp, _vp, ctypes.POINTER(ctypes.c_float), _i32, _vp, _vp, _vp,
+                               _vp, _vp, _vp],
     "sba_check_device_status": [_vp, _vp, _vp],
     "sba_debug_timeout_probe": [_vp, _vp, ctypes.c_uint64, _vp],
     "sba_perm_export": [_vp, ctypes.POINTER(ctypes.c_int32)],
@@ -153,6 +156,16 @@ def sba_build_mask(plan: int, qt, kt, top_p: Sequence[float], top_k: int, bitmas
     _check(_lib.sba_build_mask(plan, _ptr(qt), _ptr(kt), arr, int(top_k), _ptr(bitmask),
                                _ptr(row_cnt), _ptr(row_ptr), _ptr(col_idx), _ptr(work_order),
                                _ptr(workspace), _stream(stream)), "sba_build_mask")
+
+
+def sba_build_mask_noalloc(plan: int, qt, kt, top_p: Sequence[float], top_k: int, bitmask,
+                           row_cnt, row_ptr, col_idx, work_order, stream=None) -> None:
+    """sba_build_mask without a workspace: the library's static scratch is used
+    instead (see include/sba.h for the size limit and the sharing rules)."""
+    arr = (ctypes.c_float * len(top_p))(*[float(x) for x in top_p])
+    _check(_lib.sba_build_mask_noalloc(plan, _ptr(qt), _ptr(kt), arr, int(top_k), _ptr(bitmask),
+                                       _ptr(row_cnt), _ptr(row_ptr), _ptr(col_idx),
+                                       _ptr(work_order), _stream(stream)), "sba_build_mask_noalloc")
 
 
 def sba_attention(plan: int, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse=None,

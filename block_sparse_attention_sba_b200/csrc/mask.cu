@@ -20,6 +20,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -466,4 +467,150 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------
+// Allocation-free variant of sba_build_mask.
+//
+// Some callers cannot hand the library a workspace: plugin hosts whose
+// interface passes only inputs and outputs, and services that reserve all
+// device memory at start-up and forbid any later cudaMalloc (an allocation
+// there can synchronise the device or fail under memory pressure in the middle
+// of serving). For them the pooled means and the control block live in one
+// file-scope device array that every GPU loading this library holds until the
+// process exits.
+// ------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_mask_scratch[kNoAllocScratchBytes];
+
+std::once_flag g_scratch_once[kMaxDevices];
+void* g_scratch_addr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+
+// Device address of g_mask_scratch on the current device. The lookup runs once
+// per device, on that device's first call (host code must never pass the
+// symbol itself to a kernel: on the host it only names a stand-in).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_scratch_once[dev], [dev] {
+    void* ptr = nullptr;
+    g_scratch_err[dev] = cudaGetSymbolAddress(&ptr, g_mask_scratch);
+    g_scratch_addr[dev] = g_scratch_err[dev] == cudaSuccess ? ptr : nullptr;
+  });
+  *out = g_scratch_addr[dev];
+  return g_scratch_err[dev];
+}
+
+size_t noalloc_scratch_need(const sba_plan* p) {
+  const size_t pooled = (static_cast<size_t>(p->info.rows) * p->g.d * sizeof(float) + 255) & ~size_t(255);
+  return sizeof(Ctrl) + 2 * pooled;
+}
+
+// The same four launches as launch_build_mask, with the scratch pointers given.
+cudaError_t launch_build_mask_scratch(const sba_plan* p, const void* qt, const void* kt,
+                                      const float* top_p, int top_k, uint32_t* bitmask,
+                                      int32_t* row_cnt, int32_t* row_ptr, int32_t* col_idx,
+                                      int32_t* work_order, char* scratch, cudaStream_t st) {
+  KGeom g = make_kgeom(p);
+  const size_t pooled = (static_cast<size_t>(p->info.rows) * p->g.d * sizeof(float) + 255) & ~size_t(255);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(scratch);
+  float* qbar = reinterpret_cast<float*>(scratch + sizeof(Ctrl));
+  float* kbar = reinterpret_cast<float*>(scratch + sizeof(Ctrl) + pooled);
+  const int BH = g.B * g.H;
+  // the control block keeps the previous call's contents: start from zero
+  cudaError_t e = cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), st);
+  if (e != cudaSuccess) return e;
+  dim3 pg(g.nb, BH, 2);
+  if (p->g.dtype == SBA_BF16)
+    pool_kernel<__nv_bfloat16><<<pg, kPoolThreads, 0, st>>>(g, static_cast<const char*>(qt),
+                                                            static_cast<const char*>(kt), qbar, kbar);
+  else
+    pool_kernel<float><<<pg, kPoolThreads, 0, st>>>(g, static_cast<const char*>(qt),
+                                                    static_cast<const char*>(kt), qbar, kbar);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int nkp = 32;
+  while (nkp < g.nb) nkp <<= 1;
+  const size_t sel_smem = select_smem_bytes(g.d, nkp);
+  if (sel_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sel_smem));
+    if (e != cudaSuccess) return e;
+  }
+  SelectArgs sa;
+  for (int h = 0; h < 256; ++h) sa.top_p[h] = h < g.H ? top_p[h] : 1.0f;
+  dim3 sg((g.nb + kRQ - 1) / kRQ, BH);
+  select_kernel<<<sg, kSelThreads, sel_smem, st>>>(g, qbar, kbar, sa, top_k, nkp, bitmask, row_cnt);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int R = p->info.rows;
+  const size_t scan_smem = (static_cast<size_t>(kScanWarps) + 2) * (g.nb + 1) * sizeof(int);
+  if (scan_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(scan_smem));
+    if (e != cudaSuccess) return e;
+  }
+  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, g.nb, row_cnt, row_ptr, work_order,
+                                                        &ctrl->status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  expand_kernel<<<(R + 7) / 8, 256, 0, st>>>(R, g.nb, bitmask, row_ptr, col_idx);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 }  // namespace sba
+
+extern "C" sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* qt, const void* kt,
+                                             const float* top_p, int32_t top_k, uint32_t* bitmask,
+                                             int32_t* row_cnt, int32_t* row_ptr, int32_t* col_idx,
+                                             int32_t* work_order, void* stream) {
+  using namespace sba;
+  if (!plan || !qt || !kt || !top_p || !bitmask || !row_cnt || !row_ptr || !col_idx || !work_order) {
+    set_error("sba_build_mask_noalloc: NULL argument");
+    return SBA_ERR_INVALID_ARG;
+  }
+  if ((reinterpret_cast<uintptr_t>(qt) | reinterpret_cast<uintptr_t>(kt)) & 15u) {
+    set_error("qt and kt must be 16-byte aligned");
+    return SBA_ERR_INVALID_ARG;
+  }
+  if (top_k < 0) {
+    set_error("top_k must be >= 0");
+    return SBA_ERR_INVALID_ARG;
+  }
+  for (int h = 0; h < plan->g.H; ++h) {
+    const float p = top_p[h];
+    if (!(p > 0.0f) || !(p <= 1.0f)) {
+      set_error("top_p[%d] = %g; must lie in (0, 1]", h, (double)p);
+      return SBA_ERR_INVALID_ARG;
+    }
+  }
+  const size_t need = noalloc_scratch_need(plan);
+  if (need > kNoAllocScratchBytes) {
+    set_error("sba_build_mask_noalloc needs %zu bytes of scratch (2*B*H*nb*d floats + 256) but "
+              "its static scratch holds %zu; use sba_build_mask with a workspace",
+              need, kNoAllocScratchBytes);
+    return SBA_ERR_CAPACITY;
+  }
+  void* scratch = nullptr;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess || !scratch) {
+    set_error("cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    return SBA_ERR_CUDA;
+  }
+  e = launch_build_mask_scratch(plan, qt, kt, top_p, top_k, bitmask, row_cnt, row_ptr, col_idx,
+                                work_order, static_cast<char*>(scratch),
+                                static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    set_error("sba_build_mask_noalloc launch: %s", cudaGetErrorString(e));
+    return SBA_ERR_CUDA;
+  }
+  return SBA_OK;
+}

@@ -150,6 +150,29 @@ SBA_API sba_status sba_build_mask(const sba_plan* plan, const void* qt, const vo
                           int32_t* col_idx, int32_t* work_order,
                           void* workspace, void* stream);
 
+/* Allocation-free sba_build_mask (the paper has no counterpart: this is a
+ * deployment convenience). Same inputs, outputs and results as sba_build_mask,
+ * but no workspace argument: its scratch (the pooled block means and a
+ * 256-byte control block) lives in one 32 MiB array of static device memory
+ * inside the library, which every GPU that loads libsba holds until the
+ * process exits. For callers that cannot allocate device memory or carry a
+ * workspace: plugin interfaces that pass only inputs and outputs, and services
+ * that reserve all device memory at start-up and forbid cudaMalloc afterwards.
+ * Limit: 2*B*H*nb*d*4 bytes (rounded up to 256 each) + 256 <= 32 MiB, i.e.
+ * B*H*nb*d <= ~4.19 million (the Wan and HunyuanVideo-shaped layers fit);
+ * larger plans return SBA_ERR_CAPACITY before anything is launched.
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress (make that first call before any stream capture).
+ * Each call clears the control block with cudaMemsetAsync and overwrites the
+ * pooled means; the array keeps the last call's contents. All calls share the
+ * one array, so calls that overlap on the GPU (other streams, other threads)
+ * race: serialise them. Never calls cudaMalloc, cudaFree or any allocating
+ * routine. */
+SBA_API sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* qt, const void* kt,
+                                          const float* top_p, int32_t top_k,
+                                          uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
+                                          int32_t* col_idx, int32_t* work_order, void* stream);
+
 /* Block-sparse attention forward (FVAttn abstract: attention over the
  * materialised mask). For every real query slot q of block i:
  *   o_q = sum_{j in cols(i)} sum_{real keys k of j} softmax(q.k / sqrt(d)) v_k
