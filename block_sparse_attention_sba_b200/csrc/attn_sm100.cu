@@ -13,12 +13,24 @@
 //                      back over S in TMEM
 //   O += P V_j         tcgen05.mma with A = P from TMEM, B = V_j (smem,
 //                      MN-major), fp32 accumulator in TMEM
-// Warp roles (192 threads, one CTA per SM):
-//   warps 0-3  softmax + epilogue (thread t owns TMEM lane / query row t)
-//   warp  4    producer: fetches work items, TMA-loads Q and the K/V tiles into
-//              a ring of shared-memory slots in the order the MMAs use them
-//              (K0, K1, V0, K2, V1, ...)
-//   warp  5    MMA issuer (one thread) and TMEM owner
+// Issuing a tcgen05.mma blocks the issuing thread at the tensor core's pace,
+// and every commit / wait costs that thread tens of cycles, so one thread that
+// alternates S and P.V products leaves the tensor core idle whenever it waits
+// for the softmax. Two issuer warps keep it fed: one issues the S products up
+// to three key blocks ahead (three S buffers in TMEM), the other issues P.V as
+// soon as a block's P is ready.
+// Warp roles (one CTA per SM):
+//   warps 0 .. 4*NWG-1   softmax + epilogue in NWG column groups: warp w owns
+//                        TMEM lanes 32*(w%4).. (query rows) and group w/4 owns
+//                        bs/NWG columns of S and d/NWG columns of O; the
+//                        groups combine their partial row maxima through
+//                        shared memory once per key block
+//   warp  4*NWG          producer: fetches work items; TMA-loads Q, the K
+//                        tiles (ring of NK slots) and the V tiles (ring of NV
+//                        slots), K running up to two blocks ahead of V
+//   warp  4*NWG+1        S issuer (one thread) and TMEM owner
+//   warp  4*NWG+2        P.V issuer (one thread)
+// TMEM: S buffers at columns 0, 128, 256; O at 384.
 // Rescaling of O is skipped while the running row max grows by less than
 // 2^8 (the final normalisation uses the same reference max, so the result is
 // exact up to rounding); padding keys of edge cubes are masked to -inf.
@@ -40,31 +52,44 @@ namespace sba {
 namespace {
 
 constexpr int kSmemLimit = 232448;  // 227 KB: opt-in shared memory per CTA
-constexpr int kThreads = 192;
 
 template <int D, int BS>
 struct Cfg {
   static constexpr int M = 128;
+  // softmax column groups: 2 (measured best for 128x128 tiles: 64 S columns
+  // and 64 O columns per thread; 4 groups cost more in exchange and polling)
+  static constexpr int NWG = 2;
+  static constexpr int CPW = BS / NWG;  // S columns per group
+  static constexpr int DPW = D / NWG;   // O columns per group
+  static constexpr int SM_THREADS = NWG * 128;
+  static constexpr int THREADS = SM_THREADS + 96;
+  static constexpr int WARP_PROD = NWG * 4, WARP_SISS = NWG * 4 + 1, WARP_PVISS = NWG * 4 + 2;
+  static_assert(CPW % 32 == 0 && DPW % 32 == 0, "column groups must be multiples of 32");
+  static constexpr int NSB = 3;          // S buffers in TMEM
   static constexpr int PANELS = D / 64;  // 128-byte column panels along d
   static constexpr int Q_BYTES = M * D * 2;
   static constexpr int TILE_BYTES = BS * D * 2;
-  static constexpr int CTRL_BYTES = 1024;
-  static constexpr int NSLOT_RAW = (kSmemLimit - 1024 - CTRL_BYTES - Q_BYTES) / TILE_BYTES;
-  static constexpr int NSLOT = NSLOT_RAW > 8 ? 8 : NSLOT_RAW;
-  static constexpr int SMEM_USED = 1024 + Q_BYTES + NSLOT * TILE_BYTES + CTRL_BYTES;
+  static constexpr int CTRL_BYTES = 10240;  // barriers, ring, masks, row-max exchange
+  static constexpr int NT_RAW = (kSmemLimit - 1024 - CTRL_BYTES - Q_BYTES) / TILE_BYTES;
+  static constexpr int NT = NT_RAW > 8 ? 8 : NT_RAW;  // K + V slots
+  static constexpr int NK = (NT + 1) / 2, NV = NT - NK;
+  static constexpr int SMEM_USED = 1024 + Q_BYTES + NT * TILE_BYTES + CTRL_BYTES;
   // Request at least 120 KB so that only one CTA (one 512-column TMEM
   // allocation) is ever resident per SM.
   static constexpr int SMEM = SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(M, BS, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(M, D, 0, 1);
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S1 = 128, COL_O = 256;
+  static constexpr uint32_t COL_O = 384;
   // barrier indices
-  static constexpr int B_QF = 0, B_QE = 1, B_SF = 2, B_SE = B_SF + NSLOT, B_S = B_SE + NSLOT,
-                       B_P = B_S + 2, B_OD = B_P + 2, B_OF = B_OD + 1, B_OE = B_OF + 1,
-                       B_IF = B_OE + 1, B_IE = B_IF + 2, B_DR = B_IE + 2, NBAR = B_DR + 1;
-  static_assert(NSLOT >= 2, "need at least two K/V slots");
-  static_assert(NBAR * 8 <= 256, "barrier area");
+  static constexpr int B_QF = 0, B_QE = 1, B_KF = 2, B_KE = B_KF + NK, B_VF = B_KE + NK,
+                       B_VE = B_VF + NV, B_SR = B_VE + NV, B_PR = B_SR + NSB, B_PD = B_PR + NSB,
+                       B_OF = B_PD + NSB, B_OE = B_OF + 1, B_IF = B_OE + 1, B_IE = B_IF + 2,
+                       B_X = B_IE + 2, B_L = B_X + NSB, B_DR = B_L + 1, NBAR = B_DR + 2;
+  static_assert(NK >= 2 && NV >= 1, "need K and V slots");
+  static_assert(D <= 128 && BS <= 128, "TMEM plan assumes d, bs <= 128");
+  static_assert(NBAR * 8 <= 512, "barrier area");
+  static_assert(1024 + (NSB * NWG + NWG) * 128 * 4 <= CTRL_BYTES, "control area");
   static_assert(SMEM <= kSmemLimit, "shared memory budget");
 };
 
@@ -83,27 +108,6 @@ struct AttnParams {
   float scale_log2;
 };
 
-// Tile t of an item with n key blocks, in MMA consumption order:
-// K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1).
-__device__ __forceinline__ void tile_of(int t, int n, int& is_v, int& blk) {
-  if (t == 0) {
-    is_v = 0;
-    blk = 0;
-  } else if (t & 1) {
-    const int kb = (t + 1) >> 1;
-    if (kb < n) {
-      is_v = 0;
-      blk = kb;
-    } else {
-      is_v = 1;
-      blk = n - 1;
-    }
-  } else {
-    is_v = 1;
-    blk = (t >> 1) - 1;
-  }
-}
-
 // Wait that ignores the abort flag (used to drain in-flight async work).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t budget_ns,
                                                 uint32_t* status) {
@@ -120,7 +124,7 @@ __device__ __forceinline__ int block_type(const KGeom& g, int j) {
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
   using C = Cfg<D, BS>;
@@ -128,14 +132,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sQ = sm;
-  unsigned char* sSlots = sm + C::Q_BYTES;
-  unsigned char* ctl = sSlots + C::NSLOT * C::TILE_BYTES;
+  unsigned char* sK = sm + C::Q_BYTES;
+  unsigned char* sV = sK + C::NK * C::TILE_BYTES;
+  unsigned char* ctl = sV + C::NV * C::TILE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 256);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 260);
-  int* ring = reinterpret_cast<int*>(ctl + 272);        // [2][4]
-  uint32_t* emask = reinterpret_cast<uint32_t*>(ctl + 320);  // [8][4]
-  int* efull = reinterpret_cast<int*>(ctl + 448);            // [8]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 512);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 516);
+  int* ring = reinterpret_cast<int*>(ctl + 528);             // [2][4]
+  uint32_t* emask = reinterpret_cast<uint32_t*>(ctl + 576);  // [8][4]
+  int* efull = reinterpret_cast<int*>(ctl + 704);            // [8]
+  float* xmax = reinterpret_cast<float*>(ctl + 1024);        // [NSB][NWG][128] partial row maxima
+  float* xsum = xmax + C::NSB * C::NWG * 128;                // [NWG][128] partial row sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const KGeom& g = P.g;
@@ -146,26 +153,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_QF), 1);
     mbar_init(bar(C::B_QE), 1);
-    for (int s = 0; s < C::NSLOT; ++s) {
-      mbar_init(bar(C::B_SF + s), 1);
-      mbar_init(bar(C::B_SE + s), 1);
+    for (int s = 0; s < C::NK; ++s) {
+      mbar_init(bar(C::B_KF + s), 1);
+      mbar_init(bar(C::B_KE + s), 1);
+    }
+    for (int s = 0; s < C::NV; ++s) {
+      mbar_init(bar(C::B_VF + s), 1);
+      mbar_init(bar(C::B_VE + s), 1);
+    }
+    for (int b = 0; b < C::NSB; ++b) {
+      mbar_init(bar(C::B_SR + b), 1);
+      mbar_init(bar(C::B_PR + b), C::SM_THREADS);
+      mbar_init(bar(C::B_PD + b), 1);
+      mbar_init(bar(C::B_X + b), C::NWG * 4);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::B_S + b), 1);
-      mbar_init(bar(C::B_P + b), 128);
       mbar_init(bar(C::B_IF + b), 1);
-      mbar_init(bar(C::B_IE + b), 5);
+      mbar_init(bar(C::B_IE + b), 2 + C::NWG * 4);
+      mbar_init(bar(C::B_DR + b), 1);
     }
-    mbar_init(bar(C::B_OD), 1);
     mbar_init(bar(C::B_OF), 1);
-    mbar_init(bar(C::B_OE), 4);
-    mbar_init(bar(C::B_DR), 1);
+    mbar_init(bar(C::B_OE), C::NWG * 4);
+    mbar_init(bar(C::B_L), C::NWG * 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (threadIdx.x >= 32 && threadIdx.x < 40) {
     // validity masks of the 8 edge-cube types (bit 2: last in t, 1: in h, 0: in w)
-    const int ty = threadIdx.x - 32;
+    const int ty = static_cast<int>(threadIdx.x) - 32;
     const int vt = (ty & 4) ? g.T - (g.nT - 1) * g.ct : g.ct;
     const int vh = (ty & 2) ? g.Hh - (g.nH - 1) * g.ch : g.ch;
     const int vw = (ty & 1) ? g.W - (g.nW - 1) * g.cw : g.cw;
@@ -177,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < 4; ++k) emask[ty * 4 + k] = w[k];
     efull[ty] = (vt == g.ct && vh == g.ch && vw == g.cw) ? 1 : 0;
   }
-  if (warp == 5) {
+  if (warp == C::WARP_SISS) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -186,14 +201,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  // lane 0 waits, the warp follows
+  auto wait1 = [&](int b, uint32_t parity) -> bool {
+    int w = 0;
+    if (lane == 0) w = mbar_wait(bar(b), parity, budget, abort_flag, status);
+    return __shfl_sync(0xffffffffu, w, 0) != 0;
+  };
+
+  if (warp == C::WARP_PROD) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    uint32_t items = 0, tiles = 0, qloads = 0;
+    uint32_t items = 0, kt = 0, vt = 0, qloads = 0;
     bool ok = true;
     while (ok) {
       int row = -1;
@@ -222,9 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int rs = items & 1;
       if (items >= 2) {
-        int w = 0;
-        if (lane == 0) w = mbar_wait(bar(C::B_IE + rs), ((items >> 1) - 1) & 1, budget, abort_flag, status);
-        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        ok = wait1(C::B_IE + rs, ((items >> 1) - 1) & 1);
         if (!ok) break;
       }
       if (lane == 0) {
@@ -240,9 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
       const int rows_base = static_cast<int>(bh) * g.Npad;
       if (qloads >= 1) {
-        int w = 0;
-        if (lane == 0) w = mbar_wait(bar(C::B_QE), (qloads - 1) & 1, budget, abort_flag, status);
-        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        ok = wait1(C::B_QE, (qloads - 1) & 1);
         if (!ok) break;
       }
       if (lane == 0) {
@@ -252,10 +270,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                       bar(C::B_QF));
       }
       ++qloads;
+      // K runs up to NSB-1 blocks ahead of V (the S issuer works that far ahead)
+      int nk = 0, nv = 0;
       int ck = 0, cv = 0, ckb = -32, cvb = -32;
-      for (int t = 0; t < 2 * n; ++t) {
-        int isv, blk;
-        tile_of(t, n, isv, blk);
+      while (nv < n) {
+        const bool isv = !(nk < n && nk <= nv + (C::NSB - 1));
+        const int blk = isv ? nv : nk;
         const int cb = blk & ~31;
         int j;
         if (!isv) {
@@ -275,86 +295,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) atomicOr(status, kStatusCheck);
           j = 0;
         }
-        const int s = static_cast<int>(tiles % C::NSLOT);
-        const uint32_t r = tiles / C::NSLOT;
+        const uint32_t cnt = isv ? vt : kt;
+        const int nslot = isv ? C::NV : C::NK;
+        const int s = static_cast<int>(cnt % nslot);
+        const uint32_t r = cnt / nslot;
+        const int bfull = (isv ? C::B_VF : C::B_KF) + s, bempty = (isv ? C::B_VE : C::B_KE) + s;
         if (r >= 1) {
-          int w = 0;
-          if (lane == 0) w = mbar_wait(bar(C::B_SE + s), (r - 1) & 1, budget, abort_flag, status);
-          ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+          ok = wait1(bempty, (r - 1) & 1);
           if (!ok) break;
         }
         if (lane == 0) {
-          const uint32_t dst = smem_u32(sSlots + s * C::TILE_BYTES);
-          mbar_arrive_expect_tx(bar(C::B_SF + s), C::TILE_BYTES);
+          const uint32_t dst = smem_u32((isv ? sV : sK) + s * C::TILE_BYTES);
+          mbar_arrive_expect_tx(bar(bfull), C::TILE_BYTES);
           for (int p = 0; p < C::PANELS; ++p)
-            tma_load_2d(dst + p * BS * 128, isv ? &tmV : &tmK, p * 64, rows_base + j * BS,
-                        bar(C::B_SF + s));
+            tma_load_2d(dst + p * BS * 128, isv ? &tmV : &tmK, p * 64, rows_base + j * BS, bar(bfull));
         }
-        ++tiles;
+        if (isv) {
+          ++vt;
+          ++nv;
+        } else {
+          ++kt;
+          ++nk;
+        }
       }
     }
     if (*abort_flag && lane == 0) {
       // let every TMA load this CTA issued land before shared memory goes away
-      for (int s = 0; s < C::NSLOT; ++s) {
-        const uint32_t uses = tiles / C::NSLOT + (static_cast<uint32_t>(s) < tiles % C::NSLOT ? 1u : 0u);
-        if (uses) mbar_wait_drain(bar(C::B_SF + s), (uses - 1) & 1, budget, status);
+      for (int s = 0; s < C::NK; ++s) {
+        const uint32_t uses = kt / C::NK + (static_cast<uint32_t>(s) < kt % C::NK ? 1u : 0u);
+        if (uses) mbar_wait_drain(bar(C::B_KF + s), (uses - 1) & 1, budget, status);
+      }
+      for (int s = 0; s < C::NV; ++s) {
+        const uint32_t uses = vt / C::NV + (static_cast<uint32_t>(s) < vt % C::NV ? 1u : 0u);
+        if (uses) mbar_wait_drain(bar(C::B_VF + s), (uses - 1) & 1, budget, status);
       }
       if (qloads) mbar_wait_drain(bar(C::B_QF), (qloads - 1) & 1, budget, status);
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
-    uint32_t items = 0, tiles = 0, sblocks = 0, qloads = 0, ouses = 0;
+  } else if (warp == C::WARP_SISS) {
+    // ------------------------------------------------------------ S issuer
+    uint32_t items = 0, kc = 0, gs = 0, qloads = 0;
     bool ok = true;
-    auto wait1 = [&](int b, uint32_t parity) -> bool {
-      int w = 0;
-      if (lane == 0) w = mbar_wait(bar(b), parity, budget, abort_flag, status);
-      return __shfl_sync(0xffffffffu, w, 0) != 0;
-    };
     const uint32_t q_addr = smem_u32(sQ);
-    auto issue_S = [&]() -> bool {
-      const int s = static_cast<int>(tiles % C::NSLOT);
-      if (!wait1(C::B_SF + s, (tiles / C::NSLOT) & 1)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t sb = sblocks & 1;
-        const uint32_t dS = tmem + (sb ? C::COL_S1 : 0u);
-        const uint32_t k_addr = smem_u32(sSlots + s * C::TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * (C::M * 128) + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(k_addr + (kk >> 2) * (BS * 128) + off, 16, 1024);
-          mma_ss(dS, a, b, C::IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(C::B_S + sb));
-        mma_commit(bar(C::B_SE + s));
-      }
-      __syncwarp();
-      ++tiles;
-      ++sblocks;
-      return true;
-    };
-    auto issue_PV = [&](uint32_t gblk, bool first) -> bool {
-      const uint32_t sb = gblk & 1;
-      if (!wait1(C::B_P + sb, (gblk >> 1) & 1)) return false;
-      const int s = static_cast<int>(tiles % C::NSLOT);
-      if (!wait1(C::B_SF + s, (tiles / C::NSLOT) & 1)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t aP = tmem + (sb ? C::COL_S1 : 0u);
-        const uint32_t v_addr = smem_u32(sSlots + s * C::TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk) {
-          const uint64_t b = smem_desc_sw128(v_addr + kk * 2048, BS * 128, 1024);
-          mma_ts(tmem + C::COL_O, aP + kk * 8, b, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(C::B_OD));
-        mma_commit(bar(C::B_SE + s));
-      }
-      __syncwarp();
-      ++tiles;
-      return true;
-    };
     while (ok) {
       const int rs = items & 1;
       ok = wait1(C::B_IF + rs, (items >> 1) & 1);
@@ -368,19 +349,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait1(C::B_QF, qloads & 1);
       ++qloads;
       if (!ok) break;
-      tc_fence_after();
-      const uint32_t pbase = sblocks;
-      if (!issue_S()) { ok = false; break; }
-      if (n == 1 && lane == 0) mma_commit(bar(C::B_QE));
       for (int i = 0; i < n; ++i) {
-        if (i + 1 < n) {
-          if (!issue_S()) { ok = false; break; }
-          if (i + 2 == n && lane == 0) mma_commit(bar(C::B_QE));
+        const int b = static_cast<int>(gs % C::NSB);
+        if (gs >= static_cast<uint32_t>(C::NSB)) {
+          // buffer b still holds P of block gs-NSB until its P.V is done
+          ok = wait1(C::B_PD + b, (gs / C::NSB - 1) & 1);
+          if (!ok) break;
         }
+        const int s = static_cast<int>(kc % C::NK);
+        ok = wait1(C::B_KF + s, (kc / C::NK) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t dS = tmem + static_cast<uint32_t>(b) * 128u;
+          const uint32_t k_addr = smem_u32(sK + s * C::TILE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * (C::M * 128) + off, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(k_addr + (kk >> 2) * (BS * 128) + off, 16, 1024);
+            mma_ss(dS, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_SR + b));
+          mma_commit(bar(C::B_KE + s));
+          if (i == n - 1) mma_commit(bar(C::B_QE));
+        }
+        __syncwarp();
+        ++kc;
+        ++gs;
+      }
+    }
+    if (*abort_flag && lane == 0) {
+      mma_commit(bar(C::B_DR + 0));
+      mbar_wait_drain(bar(C::B_DR + 0), 0, budget, status);
+    }
+  } else if (warp == C::WARP_PVISS) {
+    // ------------------------------------------------------------ P.V issuer
+    uint32_t items = 0, vc = 0, gp = 0, ouses = 0;
+    bool ok = true;
+    while (ok) {
+      const int rs = items & 1;
+      ok = wait1(C::B_IF + rs, (items >> 1) & 1);
+      if (!ok) break;
+      const int row = ring[rs * 4 + 0], n = ring[rs * 4 + 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_IE + rs));
+      ++items;
+      if (row < 0) break;
+      if (n == 0) continue;
+      for (int i = 0; i < n; ++i) {
+        const int b = static_cast<int>(gp % C::NSB);
+        ok = wait1(C::B_PR + b, (gp / C::NSB) & 1);
+        if (!ok) break;
+        const int s = static_cast<int>(vc % C::NV);
+        ok = wait1(C::B_VF + s, (vc / C::NV) & 1);
+        if (!ok) break;
         if (i == 0 && ouses >= 1) {
-          if (!wait1(C::B_OE, (ouses - 1) & 1)) { ok = false; break; }
+          // the epilogue of the previous item has read O out of TMEM
+          ok = wait1(C::B_OE, (ouses - 1) & 1);
+          if (!ok) break;
         }
-        if (!issue_PV(pbase + i, i == 0)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t aP = tmem + static_cast<uint32_t>(b) * 128u;
+          const uint32_t v_addr = smem_u32(sV + s * C::TILE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BS / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, BS * 128, 1024);
+            mma_ts(tmem + C::COL_O, aP + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_PD + b));
+          mma_commit(bar(C::B_VE + s));
+        }
+        __syncwarp();
+        ++vc;
+        ++gp;
       }
       if (!ok) break;
       if (lane == 0) mma_commit(bar(C::B_OF));
@@ -388,20 +431,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++ouses;
     }
     if (*abort_flag && lane == 0) {
-      mma_commit(bar(C::B_DR));
-      mbar_wait_drain(bar(C::B_DR), 0, budget, status);
+      mma_commit(bar(C::B_DR + 1));
+      mbar_wait_drain(bar(C::B_DR + 1), 0, budget, status);
     }
   } else {
     // ------------------------------------------------ softmax + epilogue
-    const int t = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    constexpr int CPW = C::CPW, DPW = C::DPW, NWG = C::NWG, NSB = C::NSB;
+    const int t = static_cast<int>(threadIdx.x) & 127;  // query row == TMEM lane
+    const int wg = warp >> 2;                             // column group
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = P.scale_log2;
-    uint32_t items = 0, sblocks = 0, pvs = 0, ouses = 0;
+    auto wwait = [&](int b, uint32_t parity) -> bool {
+      const bool w = mbar_wait(bar(b), parity, budget, abort_flag, status);
+      return __all_sync(0xffffffffu, w);
+    };
+    uint32_t items = 0, gsm = 0, ouses = 0;
     bool ok = true;
     while (ok) {
       const int rs = items & 1;
-      ok = mbar_wait(bar(C::B_IF + rs), (items >> 1) & 1, budget, abort_flag, status);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = wwait(C::B_IF + rs, (items >> 1) & 1);
       if (!ok) break;
       const int row = ring[rs * 4 + 0], n = ring[rs * 4 + 1], start = ring[rs * 4 + 2];
       __syncwarp();
@@ -414,126 +462,179 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qtype = block_type(g, static_cast<int>(iq));
       const bool qvalid = (t < BS) && ((emask[qtype * 4 + (t >> 5)] >> (t & 31)) & 1u);
       const int64_t orow = static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(iq) * BS + t;
-      __nv_bfloat16* optr = P.ot + orow * D;
+      __nv_bfloat16* optr = P.ot + orow * D + wg * DPW;
       if (n == 0) {
         if (t < BS) {
-          for (int c = 0; c < D; c += 8)
+          for (int c = 0; c < DPW; c += 8)
             *reinterpret_cast<uint4*>(optr + c) = make_uint4(0u, 0u, 0u, 0u);
-          if (P.lse) P.lse[orow] = qvalid ? -INFINITY : 0.f;
+          if (P.lse && wg == 0) P.lse[orow] = qvalid ? -INFINITY : 0.f;
         }
       } else {
-        float m = -INFINITY, l = 0.f;
+        float m = -INFINITY, l = 0.f;  // l: this group's share of the row sum
         int jn = __ldg(&P.col_idx[start]);
         for (int i = 0; i < n; ++i) {
           const int j = (jn < 0 || jn >= g.nb) ? 0 : jn;
           if (i + 1 < n) jn = __ldg(&P.col_idx[start + i + 1]);
-          const uint32_t sb = sblocks & 1;
-          ok = mbar_wait(bar(C::B_S + sb), (sblocks >> 1) & 1, budget, abort_flag, status);
-          ok = __all_sync(0xffffffffu, ok);
+          const int b = static_cast<int>(gsm % NSB);
+          const uint32_t ph = (gsm / NSB) & 1;
+          ok = wwait(C::B_SR + b, ph);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t scol = tmem + lane_off + (sb ? C::COL_S1 : 0u);
-          uint32_t sr[BS];
+          const uint32_t scol = tmem + lane_off + static_cast<uint32_t>(b) * 128u;
+          uint32_t sr[CPW];
 #pragma unroll
-          for (int c = 0; c < BS / 32; ++c)
-            tmem_ld32(scol + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          for (int c = 0; c < CPW / 32; ++c)
+            tmem_ld32(scol + wg * CPW + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
           tmem_ld_wait();
-          float s[BS];
+          float s[CPW];
 #pragma unroll
-          for (int e = 0; e < BS; ++e) s[e] = __uint_as_float(sr[e]);
+          for (int e = 0; e < CPW; ++e) s[e] = __uint_as_float(sr[e]);
           const int kt = block_type(g, j);
           if (!efull[kt]) {
 #pragma unroll
-            for (int c = 0; c < BS / 32; ++c) {
-              const uint32_t w = emask[kt * 4 + c];
+            for (int c = 0; c < CPW / 32; ++c) {
+              const uint32_t w = emask[kt * 4 + (wg * CPW) / 32 + c];
 #pragma unroll
               for (int e = 0; e < 32; ++e)
                 if (!((w >> e) & 1u)) s[c * 32 + e] = -INFINITY;
             }
           }
-          float mx = s[0];
+          // partial row max over this group's columns (independent chains)
+          float mc[4];
 #pragma unroll
-          for (int e = 1; e < BS; ++e) mx = fmaxf(mx, s[e]);
-          const float mblk = mx * sl2;
-          float m_new = m, alpha = 1.f;
-          if (i == 0) {
-            m_new = mblk;
-          } else if (mblk > m + 8.0f) {
-            m_new = mblk;
-            alpha = ex2_approx(m - m_new);
+          for (int k = 0; k < 4; ++k) mc[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+          for (int e = 8; e < CPW; e += 8) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mc[k] = fmax3(mc[k], s[e + 2 * k], s[e + 2 * k + 1]);
           }
-          if (__any_sync(0xffffffffu, i > 0 && m_new != m)) {
-            // O holds PV up to block i-1: wait for it, then rescale this row
-            ok = mbar_wait(bar(C::B_OD), (pvs + i - 1) & 1, budget, abort_flag, status);
-            ok = __all_sync(0xffffffffu, ok);
+          float* xm = xmax + (b * NWG) * 128;
+          const float pm = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+          xm[wg * 128 + t] = pm;
+          // publish this group's maximum; every group has also finished
+          // loading its S columns before anyone overwrites S with P
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::B_X + b));
+          uint32_t pk[CPW / 2];
+          float2 acc[4];
+          float alpha = 1.f;
+          // Exponentials of this group's columns against the reference max.
+          // After the first block the running max is used speculatively
+          // (the usual case: no group's maximum exceeds it by more than 2^8)
+          // while the exchange completes; the rare block that does exceed it
+          // rescales O and goes round once more with the new reference.
+          float ref = m;
+          if (i == 0) {
+            ok = wwait(C::B_X + b, ph);
+            if (!ok) break;
+            float mx = xm[t];
+#pragma unroll
+            for (int k = 1; k < NWG; ++k) mx = fmaxf(mx, xm[k * 128 + t]);
+            ref = m = mx * sl2;
+          }
+#pragma unroll 1
+          for (int pass = 0; pass < 2; ++pass) {
+            const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-ref, -ref);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < CPW / 2; ++e) {
+              const float2 x = ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+              // one pair in eight runs on the FMA pipe to offload MUFU
+              const float2 pp = ((e & 7) == 5) ? exp2_poly2(x)
+                                               : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              pk[e] = pack_bf16x2(pp.x, pp.y);
+              // row sum of the bf16 values the P.V product uses, so that each
+              // output row is an exact convex combination of V rows
+              acc[e & 3] = fadd2(acc[e & 3], make_float2(__uint_as_float(pk[e] << 16),
+                                                         __uint_as_float(pk[e] & 0xFFFF0000u)));
+            }
+            if (i == 0 || pass == 1) break;
+            ok = wwait(C::B_X + b, ph);
+            if (!ok) break;
+            float mx = xm[t];
+#pragma unroll
+            for (int k = 1; k < NWG; ++k) mx = fmaxf(mx, xm[k * 128 + t]);
+            const float mblk = mx * sl2;
+            const bool grow = mblk > m + 8.0f;
+            if (!__any_sync(0xffffffffu, grow)) break;
+            const float m_new = grow ? mblk : m;
+            alpha = grow ? ex2_approx(m - m_new) : 1.f;
+            // O holds P.V up to block i-1: wait for it, rescale this group's columns
+            const uint32_t gp = gsm - 1;
+            ok = wwait(C::B_PD + static_cast<int>(gp % NSB), (gp / NSB) & 1);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < DPW / 32; ++c) {
               uint32_t r[32];
-              tmem_ld32(tmem + lane_off + C::COL_O + c * 32, r);
+              const uint32_t oc = tmem + lane_off + C::COL_O + wg * DPW + c * 32;
+              tmem_ld32(oc, r);
               tmem_ld_wait();
 #pragma unroll
               for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-              tmem_st32(tmem + lane_off + C::COL_O + c * 32, r);
+              tmem_st32(oc, r);
             }
             tmem_st_wait();
+            ref = m = m_new;
           }
+          if (!ok) break;
+          tc_fence_after();
           l *= alpha;
-          m = m_new;
-          const float neg_m = -m;
-          float rsum = 0.f;
+          // P (bf16 pairs) over the first half of this group's S columns
+          const uint32_t pcol = scol + wg * (CPW / 2);
+          if constexpr (CPW >= 64) {
 #pragma unroll
-          for (int c = 0; c < BS / 64; ++c) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * e], sl2, neg_m));
-              const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * e + 1], sl2, neg_m));
-              rsum += p0 + p1;
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-            tmem_st32(scol + c * 32, pk);
+            for (int c = 0; c < CPW / 64; ++c)
+              tmem_st32(pcol + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
+          } else {
+            tmem_st16(pcol, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
           }
+          l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+               ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
           tmem_st_wait();
-          l += rsum;
           tc_fence_before();
-          mbar_arrive(bar(C::B_P + sb));
-          ++sblocks;
+          mbar_arrive(bar(C::B_PR + b));
+          ++gsm;
         }
         if (!ok) break;
-        ok = mbar_wait(bar(C::B_OF), ouses & 1, budget, abort_flag, status);
-        ok = __all_sync(0xffffffffu, ok);
+        ok = wwait(C::B_OF, ouses & 1);
         if (!ok) break;
         tc_fence_after();
-        uint32_t orr[D];
+        uint32_t orr[DPW];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c)
-          tmem_ld32(tmem + lane_off + C::COL_O + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&orr[c * 32]));
+        for (int c = 0; c < DPW / 32; ++c)
+          tmem_ld32(tmem + lane_off + C::COL_O + wg * DPW + c * 32,
+                    *reinterpret_cast<uint32_t(*)[32]>(&orr[c * 32]));
         tmem_ld_wait();
-        float o[D];
-#pragma unroll
-        for (int e = 0; e < D; ++e) o[e] = __uint_as_float(orr[e]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(C::B_OE));
         ++ouses;
-        pvs += n;
-        if (t < BS) {
-          const float inv = qvalid ? 1.0f / l : 0.f;
+        xsum[wg * 128 + t] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_L));
+        ok = wwait(C::B_L, (ouses - 1) & 1);
+        if (!ok) break;
+        float lt = xsum[t];
 #pragma unroll
-          for (int c = 0; c < D; c += 8) {
+        for (int k = 1; k < NWG; ++k) lt += xsum[k * 128 + t];
+        if (t < BS) {
+          const float inv = qvalid ? 1.0f / lt : 0.f;
+#pragma unroll
+          for (int c = 0; c < DPW; c += 8) {
             uint4 v;
-            v.x = pack_bf16x2(o[c + 0] * inv, o[c + 1] * inv);
-            v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
-            v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
-            v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
+            v.x = pack_bf16x2(__uint_as_float(orr[c + 0]) * inv, __uint_as_float(orr[c + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(orr[c + 2]) * inv, __uint_as_float(orr[c + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(orr[c + 4]) * inv, __uint_as_float(orr[c + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(orr[c + 6]) * inv, __uint_as_float(orr[c + 7]) * inv);
             *reinterpret_cast<uint4*>(optr + c) = v;
           }
-          if (P.lse) P.lse[orow] = qvalid ? (m * 0.69314718055994531f + logf(l)) : 0.f;
+          if (P.lse && wg == 0) P.lse[orow] = qvalid ? (m * 0.69314718055994531f + logf(lt)) : 0.f;
         }
       }
-      if (P.trace && t == 0) {
+      if (P.trace && threadIdx.x == 0) {
         P.trace[static_cast<int64_t>(row) * 3 + 0] = t_start;
         P.trace[static_cast<int64_t>(row) * 3 + 1] = globaltimer_ns();
         P.trace[static_cast<int64_t>(row) * 3 + 2] = smid();
@@ -544,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == C::WARP_SISS) tmem_dealloc(tmem, C::TMEM_COLS);
   if (P.sched == SBA_SCHED_LPT && threadIdx.x == 0) {
     __threadfence();
     const uint32_t prev = atomicAdd(&P.ctrl->cta_done, 1u);
@@ -722,7 +823,7 @@ cudaError_t launch_tc(const sba_plan* p, const void* qt, const void* kt, const v
   if (e != cudaSuccess) return e;
   const int grid = ap.sched == SBA_SCHED_LPT ? std::min(sms, ap.R) : ap.R;
   if (ap.sched == SBA_SCHED_LPT) g_grid_size = grid;
-  attn_tc_kernel<D, BS><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, ap);
+  attn_tc_kernel<D, BS><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, ap);
   return cudaGetLastError();
 }
 
