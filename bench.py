@@ -47,6 +47,9 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sched-report", action="store_true")
+    ap.add_argument("--report-all", action="store_true",
+                    help="per-call timings, rooflines, density and SM idle for every workload "
+                         "(one JSON line each; not the benchmark line)")
     ap.add_argument("--gen-device", choices=["gpu", "cpu"], default="gpu",
                     help="where the synthetic inputs are generated (cpu: no GPU launches "
                          "before the timed kernels, for profiler captures)")
@@ -439,8 +442,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": mean_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": _config(wl, {"density": round(density, 4), "nnz_blocks": nnz,
-                                   "sched": "lpt-persistent"}),
+            "config": _config(wl),
+            "routing": {"density": round(density, 4), "nnz_blocks": nnz, "sched": "lpt-persistent"},
             "ms_per_call": ms_calls,
             "attention": {"tflops_tile": achieved,
                           "tflops_valid": f_valid / (attn_ms * 1e-3) / 1e12,
@@ -462,8 +465,100 @@ def run_ours(args):
     return 0
 
 
+def _alg_bytes(wl, info):
+    """Algorithmic HBM bytes of reorder (q,k,v), mask (reads qt, kt) and unreorder."""
+    e = 4 if wl.dtype == "f32" else 2
+    bh = wl.B * wl.H
+    row = wl.d * e
+    reorder = 3 * bh * (wl.N + info.Npad) * row
+    mask = 2 * bh * info.Npad * row
+    unreorder = bh * (info.Npad + wl.N) * row
+    return reorder, mask, unreorder
+
+
+def report_all(args):
+    """One JSON line per workload: per-call ms, effective TFLOPS (tile and
+    real-token FLOPs), fraction of the measured bf16 peak, HBM fractions of
+    the three bandwidth-bound calls, density and SM idle for both schedules."""
+    import torch
+
+    import block_sparse_attention_sba_b200 as sba
+    import datagen
+    dev = torch.device("cuda", 0)
+    peak, peak_sus, hbm, kind = _peaks()
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for name in ["tiny", "small", "wan", "hunyuan", "stress"]:
+        wl = datagen.WORKLOADS[name]
+        q, k, v = datagen.generate(wl, seed=0, device=dev)
+        plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+        sa = sba.SparseAttention(plan, device=dev)
+        h = plan.handle
+        o = torch.empty_like(q)
+        tp = wl.top_p_per_head()
+        R = plan.info.rows
+        trace = torch.zeros(R * 3, dtype=torch.int64, device=dev)
+        calls = {"reorder": [], "build_mask": [], "attention": [], "unreorder": []}
+        steps = 10
+        for it in range(3 + steps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            flush.zero_()
+            ev[0].record()
+            sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt)
+            ev[1].record()
+            sba.sba_build_mask(h, sa.qt, sa.kt, tp, wl.top_k, sa.bitmask, sa.row_cnt, sa.row_ptr,
+                               sa.col_idx, sa.work_order, sa.workspace)
+            ev[2].record()
+            sba.sba_attention(h, sa.qt, sa.kt, sa.vt, sa.row_ptr, sa.col_idx, sa.work_order, sa.ot,
+                              sa.lse, sba.SBA_SCHED_LPT, None, sa.workspace)
+            ev[3].record()
+            sba.sba_unreorder(h, sa.ot, o)
+            ev[4].record()
+            torch.cuda.synchronize(dev)
+            if it >= 3:
+                for i, key in enumerate(calls):
+                    calls[key].append(ev[i].elapsed_time(ev[i + 1]))
+        ms = {key: statistics.mean(val) for key, val in calls.items()}
+        nnz = int(sa.row_ptr[-1].item())
+        rc = sa.row_cnt.cpu().tolist()
+        rp = sa.row_ptr.cpu().tolist()
+        cols = sa.col_idx[:nnz].cpu().tolist()
+        lens = _block_lens(wl)
+        nb = plan.info.nb
+        f_tile = 4.0 * plan.info.bs ** 2 * wl.d * nnz
+        f_valid = sum(4.0 * wl.d * lens[r % nb] * sum(lens[j] for j in cols[rp[r]:rp[r + 1]])
+                      for r in range(R))
+        idle = {}
+        for label, mode in (("lpt", sba.SBA_SCHED_LPT), ("head_major", sba.SBA_SCHED_HEAD_MAJOR)):
+            sba.sba_attention(h, sa.qt, sa.kt, sa.vt, sa.row_ptr, sa.col_idx, sa.work_order, sa.ot,
+                              sa.lse, mode, trace, sa.workspace)
+            torch.cuda.synchronize(dev)
+            tr = trace.view(R, 3).cpu()
+            span = float(tr[:, 1].max() - tr[:, 0].min())
+            idle[label] = 1.0 - float((tr[:, 1] - tr[:, 0]).sum()) / (nsm * span)
+        rb, mb, ub = _alg_bytes(wl, plan.info)
+        att_s = ms["attention"] * 1e-3
+        line = {"workload": name, "dtype": wl.dtype, "ms": {k2: round(v2, 4) for k2, v2 in ms.items()},
+                "tflops_tile": f_tile / att_s / 1e12, "tflops_valid": f_valid / att_s / 1e12,
+                "frac_bf16_peak": f_tile / att_s / 1e12 / peak,
+                "hbm_frac": {"reorder": rb / (ms["reorder"] * 1e-3) / 1e9 / hbm,
+                             "build_mask": mb / (ms["build_mask"] * 1e-3) / 1e9 / hbm,
+                             "unreorder": ub / (ms["unreorder"] * 1e-3) / 1e9 / hbm},
+                "overhead_frac": (ms["reorder"] + ms["build_mask"] + ms["unreorder"]) / ms["attention"],
+                "density": nnz / (R * nb), "sm_idle": idle,
+                "per_head_blocks_max_over_min": float(
+                    sa.row_cnt.view(wl.B * wl.H, nb).sum(1).max() / sa.row_cnt.view(wl.B * wl.H, nb).sum(1).min()),
+                "status": sba.sba_status_string(sa.check())}
+        print(json.dumps(line), flush=True)
+        del q, k, v, sa, o, trace
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = _args()
+    if args.report_all:
+        return report_all(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -98,7 +98,7 @@ sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
   if (nb > 1024) return fail(SBA_ERR_CAPACITY, "%lld blocks per head; at most 1024", (long long)nb);
   if (G.H > 256) return fail(SBA_ERR_CAPACITY, "H = %d; at most 256", G.H);
   const int64_t BH = static_cast<int64_t>(G.B) * G.H;
-  if (BH > 65535) return fail(SBA_ERR_CAPACITY, "B*H = %lld; at most 65535", (long long)BH);
+  if (BH > 8192) return fail(SBA_ERR_CAPACITY, "B*H = %lld; at most 8192", (long long)BH);
   const int64_t R = BH * nb;
   const int64_t Npad = nb * bs;
   if (R * nb >= (1ll << 31) || BH * Npad >= (1ll << 31) || N >= (1ll << 31))

@@ -294,9 +294,13 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
 }
 
 // One CTA of 1024 threads. Dynamic shared memory: hist [kScanWarps][nb+1]
-// ints, tot [nb+1], start [nb+1].
+// ints (one bin table per warp), head totals [BH] and head ranks [BH].
+// Work order: heads by total selected blocks descending (ties: lower head
+// first), then, inside a head, rows by count descending (ties: lower row
+// first). Each warp sorts whole heads with a stable counting sort over its own
+// bin table, so the result is deterministic.
 __global__ void __launch_bounds__(kScanThreads)
-    scan_order_kernel(int R, int nb, const int32_t* __restrict__ row_cnt,
+    scan_order_kernel(int R, int nb, int BH, const int32_t* __restrict__ row_cnt,
                       int32_t* __restrict__ row_ptr, int32_t* __restrict__ work_order,
                       uint32_t* __restrict__ status) {
   extern __shared__ int ssm[];
@@ -304,9 +308,9 @@ __global__ void __launch_bounds__(kScanThreads)
   __shared__ int total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nc = nb + 1;
-  int* hist = ssm;
-  int* tot = hist + kScanWarps * nc;
-  int* start = tot + nc;
+  int* hist = ssm;                         // [kScanWarps][nc]
+  int* htot = hist + kScanWarps * nc;      // [BH]
+  int* hrank = htot + BH;                  // [BH]
 
   // ---- row_ptr: each thread owns a contiguous chunk of rows
   const int per = (R + kScanThreads - 1) / kScanThreads;
@@ -320,60 +324,78 @@ __global__ void __launch_bounds__(kScanThreads)
   }
   if (tid == 0) row_ptr[R] = total;
 
-  // ---- work order: stable counting sort by count, descending
-  for (int e = tid; e < kScanWarps * nc; e += kScanThreads) hist[e] = 0;
+  // ---- head totals (one warp per head)
+  for (int h = warp; h < BH; h += kScanWarps) {
+    int sum = 0;
+    for (int i = lane; i < nb; i += 32) sum += row_cnt[h * nb + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) htot[h] = sum;
+  }
   __syncthreads();
-  const int segl = (R + kScanWarps - 1) / kScanWarps;
-  const int s0 = min(R, warp * segl), s1 = min(R, s0 + segl);
+  // ---- head ranks: number of heads that come first
+  for (int h = tid; h < BH; h += kScanThreads) {
+    const int th = htot[h];
+    int rk = 0;
+    for (int x = 0; x < BH; ++x) {
+      const int tx = htot[x];
+      rk += (tx > th) || (tx == th && x < h);
+    }
+    hrank[h] = rk;
+  }
+  __syncthreads();
+
+  // ---- inside each head: stable counting sort by count, descending
   int* myh = hist + warp * nc;
-  for (int base = s0; base < s1; base += 32) {
-    const int r = base + lane;
-    const bool act = r < s1;
-    int c = act ? row_cnt[r] : -1;
-    if (act && (c < 0 || c > nb)) {
-      atomicOr(status, kStatusCheck);
-      c = 0;
+  for (int h = warp; h < BH; h += kScanWarps) {
+    for (int c = lane; c < nc; c += 32) myh[c] = 0;
+    __syncwarp();
+    const int base_row = h * nb;
+    for (int b = 0; b < nb; b += 32) {
+      const int i = b + lane;
+      const bool act = i < nb;
+      int c = act ? row_cnt[base_row + i] : -1;
+      if (act && (c < 0 || c > nb)) {
+        atomicOr(status, kStatusCheck);
+        c = 0;
+      }
+      const unsigned m = __match_any_sync(0xffffffffu, c);
+      if (act && lane == __ffs(m) - 1) myh[c] += __popc(m);
+      __syncwarp();
     }
-    const unsigned m = __match_any_sync(0xffffffffu, c);
-    if (act && lane == __ffs(m) - 1) myh[c] += __popc(m);
-    __syncwarp();
-  }
-  __syncthreads();
-  for (int c = tid; c < nc; c += kScanThreads) {
-    int acc = 0;
-    for (int w = 0; w < kScanWarps; ++w) {
-      const int t = hist[w * nc + c];
-      hist[w * nc + c] = acc;
-      acc += t;
+    // start of each count's run = rows with a larger count: scan bins from nb down
+    const int seg = (nc + 31) / 32;
+    const int q0 = min(nc, lane * seg), q1 = min(nc, q0 + seg);
+    int ls = 0;
+    for (int q = q0; q < q1; ++q) ls += myh[nb - q];
+    int incl = ls;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
     }
-    tot[c] = acc;
-  }
-  __syncthreads();
-  // start[c] = sum of tot[c'] for c' > c: exclusive scan in descending c
-  const int per2 = (nc + kScanThreads - 1) / kScanThreads;
-  const int q0 = min(nc, tid * per2), q1 = min(nc, q0 + per2);
-  int l2 = 0;
-  for (int q = q0; q < q1; ++q) l2 += tot[nb - q];
-  int run2 = block_exclusive_scan(l2, warp_sums, &total);
-  for (int q = q0; q < q1; ++q) {
-    start[nb - q] = run2;
-    run2 += tot[nb - q];
-  }
-  __syncthreads();
-  for (int e = tid; e < kScanWarps * nc; e += kScanThreads) hist[e] += start[e % nc];
-  __syncthreads();
-  for (int base = s0; base < s1; base += 32) {
-    const int r = base + lane;
-    const bool act = r < s1;
-    int c = act ? row_cnt[r] : -1;
-    if (act && (c < 0 || c > nb)) c = 0;
-    const unsigned m = __match_any_sync(0xffffffffu, c);
-    const int rank = __popc(m & ((1u << lane) - 1u));
-    const int pos = act ? myh[c] + rank : 0;
+    int rs = incl - ls;
     __syncwarp();
-    if (act) work_order[pos] = r;
-    if (act && lane == __ffs(m) - 1) myh[c] += __popc(m);
+    for (int q = q0; q < q1; ++q) {
+      const int t = myh[nb - q];
+      myh[nb - q] = rs;
+      rs += t;
+    }
     __syncwarp();
+    const int out_base = hrank[h] * nb;
+    for (int b = 0; b < nb; b += 32) {
+      const int i = b + lane;
+      const bool act = i < nb;
+      int c = act ? row_cnt[base_row + i] : -1;
+      if (act && (c < 0 || c > nb)) c = 0;
+      const unsigned m = __match_any_sync(0xffffffffu, c);
+      const int rank = __popc(m & ((1u << lane) - 1u));
+      const int pos = act ? myh[c] + rank : 0;
+      __syncwarp();
+      if (act) work_order[out_base + pos] = base_row + i;
+      if (act && lane == __ffs(m) - 1) myh[c] += __popc(m);
+      __syncwarp();
+    }
   }
 }
 
@@ -450,7 +472,7 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
   if (e != cudaSuccess) return e;
 
   const int R = p->info.rows;
-  const size_t scan_smem = (static_cast<size_t>(kScanWarps) + 2) * (g.nb + 1) * sizeof(int);
+  const size_t scan_smem = (static_cast<size_t>(kScanWarps) * (g.nb + 1) + 2 * static_cast<size_t>(BH)) * sizeof(int);
   static thread_local int configured_scan = 0;
   if (scan_smem > 48 * 1024 && configured_scan < static_cast<int>(scan_smem)) {
     e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -458,7 +480,7 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
     if (e != cudaSuccess) return e;
     configured_scan = static_cast<int>(scan_smem);
   }
-  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, g.nb, row_cnt, row_ptr, work_order,
+  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, g.nb, BH, row_cnt, row_ptr, work_order,
                                                         &ctrl->status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -550,13 +572,13 @@ cudaError_t launch_build_mask_scratch(const sba_plan* p, const void* qt, const v
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int R = p->info.rows;
-  const size_t scan_smem = (static_cast<size_t>(kScanWarps) + 2) * (g.nb + 1) * sizeof(int);
+  const size_t scan_smem = (static_cast<size_t>(kScanWarps) * (g.nb + 1) + 2 * static_cast<size_t>(BH)) * sizeof(int);
   if (scan_smem > 48 * 1024) {
     e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(scan_smem));
     if (e != cudaSuccess) return e;
   }
-  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, g.nb, row_cnt, row_ptr, work_order,
+  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, g.nb, BH, row_cnt, row_ptr, work_order,
                                                         &ctrl->status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

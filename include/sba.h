@@ -102,7 +102,7 @@ typedef struct sba_plan sba_plan;
 
 /* Validate a geometry and build a host-side plan (no device memory, no CUDA
  * call). Supported: bs in {64, 128}; bf16 with d in {64, 128}; f32 with d = 64;
- * nb <= 1024; B*H <= 65535; H <= 256; R*nb < 2^31; strides multiples of 8
+ * nb <= 1024; B*H <= 8192; H <= 256; R*nb < 2^31; strides multiples of 8
  * elements. Returns SBA_ERR_INVALID_ARG / SBA_ERR_UNSUPPORTED /
  * SBA_ERR_CAPACITY otherwise. The plan is immutable and may be shared by
  * threads. */
@@ -139,8 +139,11 @@ SBA_API sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o, 
  *   row_ptr   int32 [R+1]; exclusive prefix sum of row_cnt
  *   col_idx   int32 [>= row_ptr[R]]; kept j of each row, ascending (size it
  *             for max_nnz, or for a bound the caller knows)
- *   work_order int32 [R]; rows by row_cnt descending, equal counts by row
- *             ascending (longest-processing-time-first order)
+ *   work_order int32 [R]; longest first, head by head: heads (b, h) by
+ *             their total selected blocks descending (ties: lower head
+ *             first), and inside each head its rows by row_cnt descending
+ *             (ties: lower row first). Rows that run together then share one
+ *             head's keys and values in L2.
  * top_p is a host array [H]; values in (0, 1] are meaningful, p >= 1 keeps
  * every block. top_k >= 0. Scores are fp32; rows whose cumulative mass at the
  * cut lies within ~1e-5 of p may differ from an fp64 evaluation. */

@@ -237,12 +237,23 @@ def build_mask(Qt: np.ndarray, Kt: np.ndarray, g: Geom, top_p, top_k: int,
             "bitmask": bitmask, "boundary": boundary, "near_tie": near_tie}
 
 
-def lpt_order(row_cnt: np.ndarray) -> np.ndarray:
-    """Work order, longest first: rows by selected-block count descending,
-    equal counts by row index ascending (FVAttn abstract: uneven per-head
-    workloads; scheduling the heaviest rows first limits the straggler tail)."""
-    row_cnt = np.asarray(row_cnt)
-    return np.lexsort((np.arange(row_cnt.size), -row_cnt)).astype(np.int64)
+def lpt_order(row_cnt: np.ndarray, nb: int) -> np.ndarray:
+    """Work order, longest first, head by head (FVAttn abstract: uneven
+    per-head workloads; doing the heaviest work first limits the straggler
+    tail). Heads (b, h) are taken by their total selected-block count,
+    descending (ties: lower head index first); inside a head, its nb rows by
+    selected-block count, descending (ties: lower row index first).
+
+    Reading: longest-first at the granularity of heads, then of rows, so the
+    rows worked on at the same time share one head's keys and values."""
+    cnt = np.asarray(row_cnt, dtype=np.int64)
+    R = cnt.size
+    BH = R // nb
+    tot = cnt.reshape(BH, nb).sum(axis=1)
+    head_rank = np.empty(BH, dtype=np.int64)
+    head_rank[np.lexsort((np.arange(BH), -tot))] = np.arange(BH)
+    rows = np.arange(R)
+    return np.lexsort((rows, -cnt, head_rank[rows // nb])).astype(np.int64)
 
 
 # ---------------------------------------------------------------------------

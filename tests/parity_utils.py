@@ -85,7 +85,7 @@ def compare_mask(gpu: dict, orc: dict, top_p, top_k: int, nb: int, H: int) -> di
     rc = gpu["row_cnt"]
     assert gpu["row_ptr"][0] == 0
     assert np.array_equal(gpu["row_ptr"][1:], np.cumsum(rc)), "row_ptr is not the scan of row_cnt"
-    assert np.array_equal(gpu["work_order"], oracle.lpt_order(rc)), "work order differs"
+    assert np.array_equal(gpu["work_order"], oracle.lpt_order(rc, nb)), "work order differs"
     words = (nb + 31) // 32
     mism = boundary = tie = 0
     for r in range(R):

@@ -78,6 +78,7 @@ def test_host_permutation_matches_oracle(sba, T, Hh, W, cube):
     (dict(dt="f32", d=128), -2),
     (dict(T=0), -1),
     (dict(H=300), -4),
+    (dict(B=40, H=256), -4),                # B*H above 8192
     (dict(T=200, Hh=64, W=64), -4),         # too many blocks per head
 ])
 def test_plan_rejects_bad_geometry(sba, kw, code):

@@ -149,12 +149,13 @@ def test_topk_floor_and_cap():
 
 def _attn_with_csr(wl, q, k, v, row_ptr, col_idx, sched=1):
     import block_sparse_attention_sba_b200 as sba
+    g = geom_of(wl)
     plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
     sa = sba.SparseAttention(plan, device=q.device)
     sba.sba_reorder(plan.handle, q, k, v, sa.qt, sa.kt, sa.vt)
     rp = torch.tensor(row_ptr, dtype=torch.int32, device=q.device)
     ci = torch.tensor(col_idx if len(col_idx) else [0], dtype=torch.int32, device=q.device)
-    wo = torch.tensor(oracle.lpt_order(np.diff(row_ptr)), dtype=torch.int32, device=q.device)
+    wo = torch.tensor(oracle.lpt_order(np.diff(row_ptr), g.nb), dtype=torch.int32, device=q.device)
     sba.sba_attention(plan.handle, sa.qt, sa.kt, sa.vt, rp, ci, wo, sa.ot, sa.lse, sched, None,
                       sa.workspace)
     torch.cuda.synchronize()

@@ -246,9 +246,17 @@ def test_build_mask_invariants_ragged():
 
 def test_lpt_order_matches_python_sort():
     rng = np.random.default_rng(9)
-    cnt = rng.integers(0, 12, size=500)
-    exp = sorted(range(500), key=lambda r: (-cnt[r], r))
-    assert oracle.lpt_order(cnt).tolist() == exp
+    nb = 20
+    cnt = rng.integers(0, 12, size=25 * nb)
+    cnt[3 * nb:4 * nb] = cnt[7 * nb:8 * nb]          # two heads with equal totals
+    tot = cnt.reshape(25, nb).sum(1)
+    exp = sorted(range(cnt.size), key=lambda r: (-tot[r // nb], r // nb, -cnt[r], r))
+    assert oracle.lpt_order(cnt, nb).tolist() == exp
+
+
+def test_lpt_order_single_head_is_plain_longest_first():
+    cnt = np.array([3, 7, 7, 1, 0, 7, 2])
+    assert oracle.lpt_order(cnt, 7).tolist() == [1, 2, 5, 0, 6, 3, 4]
 
 
 # ------------------------------------------------------------------- attention
