@@ -158,6 +158,38 @@ def _dist():
     return ws, rank, local
 
 
+def dist_init(backend: str, device=None, timeout_s: int = 120):
+    """Join the process group torchrun describes (no-op for one process).
+    Returns the torch.distributed module or None."""
+    ws, _, _ = _dist()
+    if ws <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    kw = {"timeout": datetime.timedelta(seconds=timeout_s)}
+    if device is not None:
+        kw["device_id"] = device
+    dist.init_process_group(backend, **kw)
+    return dist
+
+
+def max_over_ranks(value: float, pg, device="cpu") -> float:
+    """Max of a per-rank scalar (timings are the slowest rank's)."""
+    if pg is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """Weak scaling: every rank processes its own replica; the job's rate is
+    all ranks' FLOPs over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def _cpu_cores():
     try:
         n = len(os.sched_getaffinity(0))
@@ -294,13 +326,7 @@ def run_ours(args):
         return 1
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-        pg = dist
+    pg = dist_init("nccl", dev)
     wl = datagen.WORKLOADS[args.workload]
     gen_dev = dev if args.gen_device == "gpu" else "cpu"
     q, k, v = datagen.generate(wl, seed=0, device=gen_dev, out_device=dev)
@@ -364,11 +390,7 @@ def run_ours(args):
         per_call["attention"].append(e[2].elapsed_time(e[3]))
         per_call["unreorder"].append(e[3].elapsed_time(e[4]))
         step_ms.append(e[0].elapsed_time(e[4]))
-    mean_step = sum(step_ms) / len(step_ms)
-    if pg:
-        t = torch.tensor([mean_step], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        mean_step = float(t.item())
+    mean_step = max_over_ranks(sum(step_ms) / len(step_ms), pg, dev)
     status = sa.check(stream)
 
     # selected-block FLOPs of one step
@@ -391,7 +413,7 @@ def run_ours(args):
     achieved = f_tile / (attn_ms * 1e-3) / 1e12
     traffic = _traffic_from_profile(os.path.join(ROOT, "block_sparse_attention_sba_b200", "csrc",
                                                  "attn_sm100.cu"))
-    value = ws * f_tile / (mean_step * 1e-3) / 1e12
+    value = whole_job_tflops(f_tile, ws, mean_step)
     ms_calls = {k: round(statistics.mean(vv), 4) for k, vv in per_call.items()}
     overhead = (ms_calls["reorder"] + ms_calls["build_mask"] + ms_calls["unreorder"]) / ms_calls["attention"]
 
@@ -416,13 +438,9 @@ def run_ours(args):
             ho.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, pg, dev)
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
-        e2e = {"value": ws * f_tile / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": whole_job_tflops(f_tile, ws, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": ho.numel() * ho.element_size()}
 
