@@ -45,7 +45,12 @@ import numpy as np
 
 @dataclass(frozen=True)
 class Geom:
-    """Grid and cube geometry (FVAttn abstract: video-aware block organization)."""
+    """Grid and block geometry (FVAttn abstract: video-aware block organization).
+
+    order "cube": blocks are ct x ch x cw cubes (padding inside edge cubes).
+    order "hilbert": tokens follow a 3-D Hilbert curve over (t, h, w) and every
+    run of bs = ct*ch*cw consecutive tokens is a block; only the last block
+    can be partial (DFSAttn: Hilbert-curve token reordering)."""
 
     T: int
     Hh: int
@@ -53,6 +58,7 @@ class Geom:
     ct: int
     ch: int
     cw: int
+    order: str = "cube"
 
     @property
     def N(self):
@@ -76,6 +82,8 @@ class Geom:
 
     @property
     def nb(self):
+        if self.order == "hilbert":
+            return -(-self.N // self.bs)
         return self.nT * self.nH * self.nW
 
     @property
@@ -87,12 +95,66 @@ class Geom:
 # Video-aware block organization (FVAttn abstract)
 # ---------------------------------------------------------------------------
 
+def hilbert_index(x, y, z, bits: int) -> int:
+    """Position of point (x, y, z) of a 2^bits cube along a 3-D Hilbert curve.
+
+    J. Skilling, "Programming the Hilbert curve" (AIP Conf. Proc. 707, 2004):
+    turn the coordinates into the curve's "transposed" form by undoing the
+    reflections and axis swaps level by level from the top bit down, Gray-encode
+    across axes, then read the index off the transposed bits, top level first,
+    one bit per axis in axis order."""
+    X = [int(x), int(y), int(z)]
+    n = 3
+    M = 1 << (bits - 1)
+    Q = M
+    while Q > 1:
+        P = Q - 1
+        for i in range(n):
+            if X[i] & Q:
+                X[0] ^= P                      # reflect the low bits of axis 0
+            else:
+                t = (X[0] ^ X[i]) & P          # swap the low bits of axes 0 and i
+                X[0] ^= t
+                X[i] ^= t
+        Q >>= 1
+    for i in range(1, n):                      # Gray encode across axes
+        X[i] ^= X[i - 1]
+    t = 0
+    Q = M
+    while Q > 1:
+        if X[n - 1] & Q:
+            t ^= Q - 1
+        Q >>= 1
+    for i in range(n):
+        X[i] ^= t
+    h = 0
+    for b in range(bits - 1, -1, -1):
+        for i in range(n):
+            h = (h << 1) | ((X[i] >> b) & 1)
+    return h
+
+
+def hilbert_bits(g: Geom) -> int:
+    """Bits per axis of the smallest power-of-two cube holding the grid."""
+    side = max(g.T, g.Hh, g.W)
+    return max(1, (side - 1).bit_length())
+
+
 def slot_of_token(g: Geom) -> np.ndarray:
     """Slot of every raster token ``n = (t*Hh + h)*W + w``.
 
-    The token lands in cube ``blk = (t//ct * nH + h//ch) * nW + w//cw`` at
+    Hilbert order: slot = rank of the token's Hilbert index among all tokens.
+    Cube order: the token lands in cube ``blk = (t//ct * nH + h//ch) * nW + w//cw`` at
     in-cube offset ``((t%ct)*ch + h%ch)*cw + w%cw``; slot = blk*bs + offset.
     """
+    if g.order == "hilbert":
+        # the token's rank along the curve among the grid's tokens
+        bits = hilbert_bits(g)
+        idx = np.array([hilbert_index(t, h, w, bits) for t in range(g.T) for h in range(g.Hh)
+                        for w in range(g.W)], dtype=np.int64)
+        slot = np.empty(g.N, dtype=np.int64)
+        slot[np.argsort(idx, kind="stable")] = np.arange(g.N)
+        return slot
     t, h, w = np.meshgrid(np.arange(g.T), np.arange(g.Hh), np.arange(g.W), indexing="ij")
     t, h, w = t.ravel(), h.ravel(), w.ravel()
     blk = ((t // g.ct) * g.nH + (h // g.ch)) * g.nW + (w // g.cw)

@@ -381,3 +381,77 @@ def test_forward_on_tiny_workload_is_consistent():
     o, m, lse = oracle.forward(q, k, v, g, wl.top_p_per_head(), wl.top_k)
     assert o.shape == q.shape and np.all(np.isfinite(o))
     _mask_invariants(m, wl.top_p_per_head(), wl.top_k, g.nb)
+
+
+# ------------------------------------------------------------- Hilbert order
+# catches: broken reflections / axis swaps (non-adjacent steps), wrong bit
+# interleave (sub-cubes not contiguous), rank vs index mix-ups on ragged grids
+
+from oracle.oracle import hilbert_index
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_hilbert_curve_is_a_bijective_unit_step_walk(bits):
+    side = 1 << bits
+    pts = [(x, y, z) for x in range(side) for y in range(side) for z in range(side)]
+    idx = [hilbert_index(*p, bits) for p in pts]
+    assert sorted(idx) == list(range(side ** 3))
+    walk = [p for _, p in sorted(zip(idx, pts))]
+    assert walk[0] == (0, 0, 0)
+    for a, b in zip(walk, walk[1:]):
+        assert sum(abs(u - v) for u, v in zip(a, b)) == 1
+    end = walk[-1]  # the curve ends on a corner next to the start corner
+    assert sorted(end) == [0, 0, side - 1]
+
+
+@pytest.mark.parametrize("bits,level", [(3, 1), (3, 2), (4, 2), (4, 3)])
+def test_hilbert_aligned_subcubes_are_contiguous_runs(bits, level):
+    side, sub = 1 << bits, 1 << level
+    for x0 in range(0, side, sub):
+        for y0 in range(0, side, sub):
+            for z0 in range(0, side, sub):
+                idx = sorted(hilbert_index(x, y, z, bits) for x in range(x0, x0 + sub)
+                             for y in range(y0, y0 + sub) for z in range(z0, z0 + sub))
+                assert idx[-1] - idx[0] == sub ** 3 - 1 and idx[0] % sub ** 3 == 0
+
+
+def test_hilbert_hand_worked_example():
+    lines = [l for l in open(os.path.join(GOLDEN, "perm_worked.txt")) if not l.startswith("#")]
+    kv = {l.split(":")[0]: [int(x) for x in l.split(":")[1].split()] for l in lines if ":" in l}
+    g = Geom(*kv["hilbert_geometry"], order="hilbert")
+    assert oracle.slot_of_token(g).tolist() == kv["hilbert_slot_of_token"]
+
+
+HGEOMS = [Geom(5, 9, 7, 2, 4, 4, "hilbert"), Geom(4, 8, 8, 4, 4, 4, "hilbert"),
+          Geom(3, 10, 6, 1, 8, 8, "hilbert"), Geom(1, 1, 3, 1, 1, 2, "hilbert")]
+
+
+@pytest.mark.parametrize("g", HGEOMS, ids=str)
+def test_hilbert_slots_fill_a_prefix_and_blocks_are_runs(g):
+    s = oracle.slot_of_token(g)
+    assert sorted(s.tolist()) == list(range(g.N))      # slots [0, N): only the tail pads
+    L = oracle.block_len(g)
+    assert L[:-1].tolist() == [g.bs] * (g.nb - 1) and L[-1] == g.N - (g.nb - 1) * g.bs
+    # consecutive slots are consecutive along the curve over the enclosing cube
+    bits = oracle.oracle.hilbert_bits(g)
+    t, h, w = np.unravel_index(np.arange(g.N), (g.T, g.Hh, g.W))
+    hidx = np.array([hilbert_index(a, b, c, bits) for a, b, c in zip(t, h, w)])
+    assert np.all(np.diff(hidx[np.argsort(s)]) > 0)
+    X = np.random.default_rng(20).standard_normal((1, 2, g.N, 3))
+    assert np.array_equal(oracle.unreorder(oracle.reorder(X, g), g), X)
+
+
+def test_hilbert_pooling_and_dense_attention():
+    g = Geom(5, 9, 7, 2, 4, 4, "hilbert")
+    rng = np.random.default_rng(21)
+    C = rng.standard_normal((1, 1, g.nb, 4))
+    X = C[:, :, oracle.slot_of_token(g) // g.bs]
+    np.testing.assert_allclose(oracle.pool(oracle.reorder(X, g), g), C, atol=1e-12)
+    q, k, v = (rng.standard_normal((1, 2, g.N, 16)) for _ in range(3))
+    qt, kt, vt = (oracle.reorder(x, g) for x in (q, k, v))
+    m = oracle.build_mask(qt, kt, g, [1.0, 1.0], 1)
+    Ot, _ = oracle.attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"])
+    valid = oracle.slot_valid(g)
+    ref = _dense_sdpa(qt, kt, vt, g)
+    np.testing.assert_allclose(Ot[:, :, valid], ref[:, :, valid], atol=1e-12)
+    _mask_invariants(oracle.build_mask(qt, kt, g, [0.7, 0.9], 2), [0.7, 0.9], 2, g.nb)
