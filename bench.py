@@ -279,10 +279,10 @@ def sched_report(dev, name="stress", reps=3):
     import datagen
     wl = datagen.WORKLOADS[name]
     q, k, v = datagen.generate(wl, seed=0, device=dev)
-    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube, order=wl.order)
     sa = sba.SparseAttention(plan, device=dev)
     h = plan.handle
-    sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt)
+    sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace)
     sba.sba_build_mask(h, sa.qt, sa.kt, wl.top_p_per_head(), wl.top_k, sa.bitmask, sa.row_cnt,
                        sa.row_ptr, sa.col_idx, sa.work_order, sa.workspace)
     R = plan.info.rows
@@ -330,7 +330,7 @@ def run_ours(args):
     wl = datagen.WORKLOADS[args.workload]
     gen_dev = dev if args.gen_device == "gpu" else "cpu"
     q, k, v = datagen.generate(wl, seed=0, device=gen_dev, out_device=dev)
-    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube, order=wl.order)
     sa = sba.SparseAttention(plan, device=dev)
     h = plan.handle
     o = torch.empty_like(q)
@@ -340,7 +340,7 @@ def run_ours(args):
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt, stream)
+        sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace, stream)
         if ev:
             ev[1].record(stream)
         sba.sba_build_mask(h, sa.qt, sa.kt, top_p, wl.top_k, sa.bitmask, sa.row_cnt, sa.row_ptr,
@@ -351,7 +351,7 @@ def run_ours(args):
                           sa.lse, sba.SBA_SCHED_LPT, None, sa.workspace, stream)
         if ev:
             ev[3].record(stream)
-        sba.sba_unreorder(h, sa.ot, o, stream)
+        sba.sba_unreorder(h, sa.ot, o, sa.workspace, stream)
         if ev:
             ev[4].record(stream)
 
@@ -506,10 +506,11 @@ def report_all(args):
     peak, peak_sus, hbm, kind = _peaks()
     nsm = torch.cuda.get_device_properties(dev).multi_processor_count
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for name in ["tiny", "small", "wan", "hunyuan", "stress"]:
-        wl = datagen.WORKLOADS[name]
+    for name in ["tiny", "small", "wan", "hunyuan", "stress", "wan_hilbert"]:
+        wl = (datagen.with_order(datagen.WORKLOADS["wan"], "hilbert") if name == "wan_hilbert"
+              else datagen.WORKLOADS[name])
         q, k, v = datagen.generate(wl, seed=0, device=dev)
-        plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+        plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube, order=wl.order)
         sa = sba.SparseAttention(plan, device=dev)
         h = plan.handle
         o = torch.empty_like(q)
@@ -522,7 +523,7 @@ def report_all(args):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
             flush.zero_()
             ev[0].record()
-            sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt)
+            sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace)
             ev[1].record()
             sba.sba_build_mask(h, sa.qt, sa.kt, tp, wl.top_k, sa.bitmask, sa.row_cnt, sa.row_ptr,
                                sa.col_idx, sa.work_order, sa.workspace)
@@ -530,7 +531,7 @@ def report_all(args):
             sba.sba_attention(h, sa.qt, sa.kt, sa.vt, sa.row_ptr, sa.col_idx, sa.work_order, sa.ot,
                               sa.lse, sba.SBA_SCHED_LPT, None, sa.workspace)
             ev[3].record()
-            sba.sba_unreorder(h, sa.ot, o)
+            sba.sba_unreorder(h, sa.ot, o, sa.workspace)
             ev[4].record()
             torch.cuda.synchronize(dev)
             if it >= 3:

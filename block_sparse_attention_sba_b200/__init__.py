@@ -34,6 +34,8 @@ SBA_F32 = 0
 SBA_BF16 = 1
 SBA_SCHED_LPT = 0
 SBA_SCHED_HEAD_MAJOR = 1
+SBA_ORDER_CUBE = 0
+SBA_ORDER_HILBERT = 1
 
 EXPORTED = ["sba_plan_create", "sba_plan_destroy", "sba_plan_query", "sba_workspace_init",
             "sba_reorder", "sba_unreorder", "sba_build_mask", "sba_attention",
@@ -47,7 +49,7 @@ class sba_geometry(ctypes.Structure):
                 ("Hh", ctypes.c_int32), ("W", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("ct", ctypes.c_int32), ("ch", ctypes.c_int32), ("cw", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("sB", ctypes.c_int64), ("sH", ctypes.c_int64),
-                ("sN", ctypes.c_int64)]
+                ("sN", ctypes.c_int64), ("order", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class sba_plan_info(ctypes.Structure):
@@ -64,8 +66,8 @@ _sig = {
     "sba_plan_destroy": [_vp],
     "sba_plan_query": [_vp, ctypes.POINTER(sba_plan_info)],
     "sba_workspace_init": [_vp, _vp, _vp],
-    "sba_reorder": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
-    "sba_unreorder": [_vp, _vp, _vp, _vp],
+    "sba_reorder": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "sba_unreorder": [_vp, _vp, _vp, _vp, _vp],
     "sba_build_mask": [_vp, _vp, _vp, ctypes.POINTER(ctypes.c_float), _i32, _vp, _vp, _vp, _vp,
                        _vp, _vp, _vp],
     "sba_attention": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp],
@@ -141,13 +143,14 @@ def sba_workspace_init(plan: int, workspace, stream=None) -> None:
     _check(_lib.sba_workspace_init(plan, _ptr(workspace), _stream(stream)), "sba_workspace_init")
 
 
-def sba_reorder(plan: int, q, k, v, qt, kt, vt, stream=None) -> None:
+def sba_reorder(plan: int, q, k, v, qt, kt, vt, workspace=None, stream=None) -> None:
     _check(_lib.sba_reorder(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(qt), _ptr(kt), _ptr(vt),
-                            _stream(stream)), "sba_reorder")
+                            _ptr(workspace), _stream(stream)), "sba_reorder")
 
 
-def sba_unreorder(plan: int, ot, o, stream=None) -> None:
-    _check(_lib.sba_unreorder(plan, _ptr(ot), _ptr(o), _stream(stream)), "sba_unreorder")
+def sba_unreorder(plan: int, ot, o, workspace=None, stream=None) -> None:
+    _check(_lib.sba_unreorder(plan, _ptr(ot), _ptr(o), _ptr(workspace), _stream(stream)),
+           "sba_unreorder")
 
 
 def sba_build_mask(plan: int, qt, kt, top_p: Sequence[float], top_k: int, bitmask, row_cnt,
@@ -210,13 +213,16 @@ class Plan:
     view of q/k/v/o (d contiguous)."""
 
     def __init__(self, B: int, H: int, T: int, Hh: int, W: int, d: int, cube,
-                 dtype: str = "bf16", strides: Optional[Sequence[int]] = None):
+                 dtype: str = "bf16", strides: Optional[Sequence[int]] = None,
+                 order: str = "cube"):
         N = T * Hh * W
         if strides is None:
             strides = (H * N * d, N * d, d)
         self.geom = sba_geometry(B, H, T, Hh, W, d, cube[0], cube[1], cube[2],
                                  SBA_BF16 if dtype == "bf16" else SBA_F32,
-                                 int(strides[0]), int(strides[1]), int(strides[2]))
+                                 int(strides[0]), int(strides[1]), int(strides[2]),
+                                 SBA_ORDER_HILBERT if order == "hilbert" else SBA_ORDER_CUBE, 0)
+        self.order = order
         self.handle = sba_plan_create(self.geom)
         self.info = sba_plan_query(self.handle)
         self.B, self.H, self.T, self.Hh, self.W, self.d = B, H, T, Hh, W, d
@@ -224,12 +230,12 @@ class Plan:
         self.dtype = dtype
 
     @classmethod
-    def for_tensor(cls, q, T: int, Hh: int, W: int, cube) -> "Plan":
+    def for_tensor(cls, q, T: int, Hh: int, W: int, cube, order: str = "cube") -> "Plan":
         B, H, N, d = q.shape
         assert N == T * Hh * W and q.stride(3) == 1
         import torch
         dt = "bf16" if q.dtype == torch.bfloat16 else "f32"
-        return cls(B, H, T, Hh, W, d, cube, dt, (q.stride(0), q.stride(1), q.stride(2)))
+        return cls(B, H, T, Hh, W, d, cube, dt, (q.stride(0), q.stride(1), q.stride(2)), order)
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -257,6 +263,8 @@ class SparseAttention:
         self.work_order = mk(inf.rows, dtype=torch.int32)
         self.lse = mk(B, H, inf.Npad, dtype=torch.float32)
         self.workspace = torch.zeros(inf.workspace_bytes, dtype=torch.uint8, device=device)
+        if torch.cuda.is_available():
+            sba_workspace_init(plan.handle, self.workspace)
 
     def __call__(self, q, k, v, top_p, top_k: int, o=None, sched: int = SBA_SCHED_LPT,
                  trace=None, stream=None):
@@ -266,12 +274,12 @@ class SparseAttention:
         if o is None:
             o = torch.empty_like(q)
         top_p = list(top_p) if len(top_p) == p.H else [float(top_p[0])] * p.H
-        sba_reorder(h, q, k, v, self.qt, self.kt, self.vt, stream)
+        sba_reorder(h, q, k, v, self.qt, self.kt, self.vt, self.workspace, stream)
         sba_build_mask(h, self.qt, self.kt, top_p, top_k, self.bitmask, self.row_cnt,
                        self.row_ptr, self.col_idx, self.work_order, self.workspace, stream)
         sba_attention(h, self.qt, self.kt, self.vt, self.row_ptr, self.col_idx, self.work_order,
                       self.ot, self.lse, sched, trace, self.workspace, stream)
-        sba_unreorder(h, self.ot, o, stream)
+        sba_unreorder(h, self.ot, o, self.workspace, stream)
         return o
 
     def check(self, stream=None) -> int:

@@ -5,7 +5,10 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <new>
+#include <utility>
+#include <vector>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -39,6 +42,9 @@ KGeom make_kgeom(const sba_plan* p) {
   k.nW = p->info.nW;
   k.nb = p->info.nb;
   k.Npad = p->info.Npad;
+  k.order = G.order;
+  k.N = G.T * G.Hh * G.W;
+  k.tail = k.N - (k.nb - 1) * k.bs;
   k.sB = G.sB;
   k.sH = G.sH;
   k.sN = G.sN;
@@ -73,6 +79,57 @@ static sba_status cuda_fail(cudaError_t e, const char* what) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Position of (x, y, z) along a 3-D Hilbert curve over a 2^bits cube, after
+// J. Skilling, "Programming the Hilbert curve" (2004): undo the curve's
+// reflections and axis exchanges from the top bit down, Gray-encode across the
+// axes, then interleave the transposed bits (top level first, axes in order).
+static uint64_t hilbert3(uint32_t x, uint32_t y, uint32_t z, int bits) {
+  uint32_t X[3] = {x, y, z};
+  const uint32_t top = 1u << (bits - 1);
+  for (uint32_t q = top; q > 1; q >>= 1) {
+    const uint32_t low = q - 1;
+    for (int i = 0; i < 3; ++i) {
+      if (X[i] & q) {
+        X[0] ^= low;
+      } else {
+        const uint32_t sw = (X[0] ^ X[i]) & low;
+        X[0] ^= sw;
+        X[i] ^= sw;
+      }
+    }
+  }
+  X[1] ^= X[0];
+  X[2] ^= X[1];
+  uint32_t flip = 0;
+  for (uint32_t q = top; q > 1; q >>= 1)
+    if (X[2] & q) flip ^= q - 1;
+  for (int i = 0; i < 3; ++i) X[i] ^= flip;
+  uint64_t h = 0;
+  for (int b = bits - 1; b >= 0; --b)
+    for (int i = 0; i < 3; ++i) h = (h << 1) | ((X[i] >> b) & 1u);
+  return h;
+}
+
+// Hilbert-order tables: slot of every raster token and token of every slot.
+static void build_hilbert_tables(sba_plan* p) {
+  const sba_geometry& G = p->g;
+  const int N = G.T * G.Hh * G.W;
+  int side = std::max(G.T, std::max(G.Hh, G.W)), bits = 1;
+  while ((1 << bits) < side) ++bits;
+  std::vector<std::pair<uint64_t, int32_t>> key(N);
+  int n = 0;
+  for (int t = 0; t < G.T; ++t)
+    for (int h = 0; h < G.Hh; ++h)
+      for (int w = 0; w < G.W; ++w, ++n) key[n] = {hilbert3(t, h, w, bits), n};
+  std::sort(key.begin(), key.end());
+  p->slot_of_token.assign(N, 0);
+  p->token_of_slot.assign(p->info.Npad, -1);
+  for (int r = 0; r < N; ++r) {
+    p->slot_of_token[key[r].second] = r;
+    p->token_of_slot[r] = key[r].second;
+  }
+}
+
 extern "C" {
 
 sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
@@ -85,6 +142,9 @@ sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
     return fail(SBA_ERR_INVALID_ARG, "all sizes must be positive");
   if (G.dtype != SBA_F32 && G.dtype != SBA_BF16)
     return fail(SBA_ERR_INVALID_ARG, "dtype must be SBA_F32 or SBA_BF16");
+  if (G.order != SBA_ORDER_CUBE && G.order != SBA_ORDER_HILBERT)
+    return fail(SBA_ERR_INVALID_ARG, "order must be SBA_ORDER_CUBE or SBA_ORDER_HILBERT");
+  if (G.reserved != 0) return fail(SBA_ERR_INVALID_ARG, "reserved must be 0");
   const int64_t bs = static_cast<int64_t>(G.ct) * G.ch * G.cw;
   if (bs != 64 && bs != 128)
     return fail(SBA_ERR_UNSUPPORTED, "block size ct*ch*cw = %lld; supported: 64, 128", (long long)bs);
@@ -93,8 +153,10 @@ sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
   if (G.dtype == SBA_F32 && G.d != 64)
     return fail(SBA_ERR_UNSUPPORTED, "f32 head dim %d; supported: 64", G.d);
   const int64_t nT = (G.T + G.ct - 1) / G.ct, nH = (G.Hh + G.ch - 1) / G.ch, nW = (G.W + G.cw - 1) / G.cw;
-  const int64_t nb = nT * nH * nW;
   const int64_t N = static_cast<int64_t>(G.T) * G.Hh * G.W;
+  const int64_t nb = G.order == SBA_ORDER_HILBERT ? (N + bs - 1) / bs : nT * nH * nW;
+  if (G.order == SBA_ORDER_HILBERT && std::max(G.T, std::max(G.Hh, G.W)) > (1 << 20))
+    return fail(SBA_ERR_CAPACITY, "Hilbert order needs every grid side <= 2^20");
   if (nb > 1024) return fail(SBA_ERR_CAPACITY, "%lld blocks per head; at most 1024", (long long)nb);
   if (G.H > 256) return fail(SBA_ERR_CAPACITY, "H = %d; at most 256", G.H);
   const int64_t BH = static_cast<int64_t>(G.B) * G.H;
@@ -127,7 +189,12 @@ sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
   p->ws_qbar = 256;
   const size_t pooled = align256(static_cast<size_t>(R) * G.d * sizeof(float));
   p->ws_kbar = p->ws_qbar + pooled;
-  p->info.workspace_bytes = p->ws_kbar + pooled;
+  p->ws_perm = p->ws_kbar + pooled;
+  p->info.workspace_bytes = p->ws_perm;
+  if (G.order == SBA_ORDER_HILBERT) {
+    build_hilbert_tables(p);
+    p->info.workspace_bytes += align256(static_cast<size_t>(Npad) * sizeof(int32_t));
+  }
   p->wait_budget_ns = 4000000000ull;  // 4 s: no healthy wait comes near it
   const char* env = getenv("SBA_WAIT_BUDGET_NS");
   if (env) {
@@ -149,14 +216,29 @@ sba_status sba_plan_query(const sba_plan* plan, sba_plan_info* info) {
 sba_status sba_workspace_init(const sba_plan* plan, void* workspace, void* stream) {
   g_err[0] = '\0';
   if (!plan || !workspace) return fail(SBA_ERR_INVALID_ARG, "plan and workspace must be non-NULL");
-  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(Ctrl), static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "cudaMemsetAsync");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(Ctrl), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if (plan->g.order == SBA_ORDER_HILBERT) {
+    // from pageable host memory: returns once the table has been staged
+    e = cudaMemcpyAsync(static_cast<char*>(workspace) + plan->ws_perm, plan->token_of_slot.data(),
+                        plan->token_of_slot.size() * sizeof(int32_t), cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(permutation)");
+  }
+  return SBA_OK;
+}
+
+static const int32_t* perm_table(const sba_plan* plan, const void* workspace) {
+  if (plan->g.order != SBA_ORDER_HILBERT) return nullptr;
+  return reinterpret_cast<const int32_t*>(static_cast<const char*>(workspace) + plan->ws_perm);
 }
 
 sba_status sba_reorder(const sba_plan* plan, const void* q, const void* k, const void* v, void* qt,
-                       void* kt, void* vt, void* stream) {
+                       void* kt, void* vt, const void* workspace, void* stream) {
   g_err[0] = '\0';
   if (!plan) return fail(SBA_ERR_INVALID_ARG, "plan must be non-NULL");
+  if (plan->g.order == SBA_ORDER_HILBERT && (!workspace || !aligned16(workspace)))
+    return fail(SBA_ERR_INVALID_ARG, "Hilbert order needs the initialised workspace");
   const void* src[3] = {q, k, v};
   void* dst[3] = {qt, kt, vt};
   for (int i = 0; i < 3; ++i) {
@@ -165,17 +247,22 @@ sba_status sba_reorder(const sba_plan* plan, const void* q, const void* k, const
     if (src[i] && (!aligned16(src[i]) || !aligned16(dst[i])))
       return fail(SBA_ERR_INVALID_ARG, "tensor %d: pointers must be 16-byte aligned", i);
   }
-  cudaError_t e = launch_reorder(plan, 0, src, dst, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_reorder(plan, 0, src, dst, perm_table(plan, workspace),
+                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_reorder launch");
 }
 
-sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o, void* stream) {
+sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o, const void* workspace,
+                         void* stream) {
   g_err[0] = '\0';
   if (!plan || !ot || !o) return fail(SBA_ERR_INVALID_ARG, "plan, ot and o must be non-NULL");
+  if (plan->g.order == SBA_ORDER_HILBERT && (!workspace || !aligned16(workspace)))
+    return fail(SBA_ERR_INVALID_ARG, "Hilbert order needs the initialised workspace");
   if (!aligned16(ot) || !aligned16(o)) return fail(SBA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   const void* src[3] = {ot, nullptr, nullptr};
   void* dst[3] = {o, nullptr, nullptr};
-  cudaError_t e = launch_reorder(plan, 1, src, dst, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_reorder(plan, 1, src, dst, perm_table(plan, workspace),
+                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_unreorder launch");
 }
 
@@ -246,6 +333,10 @@ sba_status sba_debug_timeout_probe(const sba_plan* plan, void* workspace, uint64
 sba_status sba_perm_export(const sba_plan* plan, int32_t* slot_of_token) {
   if (!plan || !slot_of_token) return fail(SBA_ERR_INVALID_ARG, "plan and output must be non-NULL");
   const sba_geometry& G = plan->g;
+  if (G.order == SBA_ORDER_HILBERT) {
+    std::copy(plan->slot_of_token.begin(), plan->slot_of_token.end(), slot_of_token);
+    return SBA_OK;
+  }
   const int nH = plan->info.nH, nW = plan->info.nW, bs = plan->info.bs;
   int64_t n = 0;
   for (int t = 0; t < G.T; ++t)

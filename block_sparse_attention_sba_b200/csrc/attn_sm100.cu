@@ -115,7 +115,10 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
   return mbar_wait(bar, parity, budget_ns, &never, status);
 }
 
+// Validity class of block j: cube order, bit 2 / 1 / 0 = last cube along
+// t / h / w; Hilbert order, 1 for a partial last block, else 0.
 __device__ __forceinline__ int block_type(const KGeom& g, int j) {
+  if (g.order == SBA_ORDER_HILBERT) return (j == g.nb - 1 && g.tail < g.bs) ? 1 : 0;
   uint32_t rest, tw, tt, th;
   g.dv_nW.divmod(static_cast<uint32_t>(j), rest, tw);
   g.dv_nH.divmod(rest, tt, th);
@@ -185,12 +188,16 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
     const int vh = (ty & 2) ? g.Hh - (g.nH - 1) * g.ch : g.ch;
     const int vw = (ty & 1) ? g.W - (g.nW - 1) * g.cw : g.cw;
     uint32_t w[4] = {0u, 0u, 0u, 0u};
+    int full = 1;
     for (int c = 0; c < BS; ++c) {
       const int lt = c / (g.ch * g.cw), lh = (c / g.cw) % g.ch, lw = c % g.cw;
-      if (lt < vt && lh < vh && lw < vw) w[c >> 5] |= 1u << (c & 31);
+      const bool ok = (g.order == SBA_ORDER_HILBERT) ? (ty != 1 || c < g.tail)
+                                                    : (lt < vt && lh < vh && lw < vw);
+      if (ok) w[c >> 5] |= 1u << (c & 31);
+      else full = 0;
     }
     for (int k = 0; k < 4; ++k) emask[ty * 4 + k] = w[k];
-    efull[ty] = (vt == g.ct && vh == g.ch && vw == g.cw) ? 1 : 0;
+    efull[ty] = full;
   }
   if (warp == C::WARP_SISS) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -680,6 +687,7 @@ __global__ void __launch_bounds__(128)
   const int64_t head = static_cast<int64_t>(bh) * g.Npad;
 
   auto valid_slot = [&](int blk, int c) -> bool {
+    if (g.order == SBA_ORDER_HILBERT) return blk * BS + c < g.N;
     uint32_t rest, tw, tt, th;
     g.dv_nW.divmod(static_cast<uint32_t>(blk), rest, tw);
     g.dv_nH.divmod(rest, tt, th);

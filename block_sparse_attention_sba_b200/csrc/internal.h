@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "../../include/sba.h"
 
 struct sba_plan {
@@ -12,7 +14,10 @@ struct sba_plan {
   int esize;               // bytes per element (2 or 4)
   size_t ws_ctrl;          // offset of the control block (status, counters)
   size_t ws_qbar, ws_kbar; // offsets of the pooled means (fp32 [B*H][nb][d])
+  size_t ws_perm;          // Hilbert order: offset of token_of_slot (int32 [Npad])
   uint64_t wait_budget_ns; // bounded-wait limit for device waits
+  std::vector<int32_t> slot_of_token;  // Hilbert order: int32 [N]
+  std::vector<int32_t> token_of_slot;  // Hilbert order: int32 [Npad], -1 = padding
 };
 
 namespace sba {
@@ -51,6 +56,9 @@ struct DivMod {
 // Geometry in the form the kernels take by value.
 struct KGeom {
   int32_t B, H, T, Hh, W, d, ct, ch, cw, bs, nT, nH, nW, nb, Npad;
+  int32_t order;  // sba_order
+  int32_t N;      // tokens per head
+  int32_t tail;   // Hilbert order: real tokens in the last block
   int64_t sB, sH, sN;
   DivMod dv_cw, dv_chcw, dv_nW, dv_nH, dv_H, dv_nb;
 };
@@ -59,7 +67,7 @@ KGeom make_kgeom(const sba_plan* p);
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_reorder(const sba_plan* p, int direction, const void* src[3], void* dst[3],
-                           cudaStream_t st);
+                           const int32_t* token_of_slot, cudaStream_t st);
 cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
                               const float* top_p, int top_k, uint32_t* bitmask, int32_t* row_cnt,
                               int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,

@@ -1,6 +1,8 @@
 // reorder.cu -- video-aware block organization (FVAttn: Adaptive Sparse
 // Attention with Runtime Load Balancing for Video Generation, abstract):
-// gather raster (t, h, w) tokens into spatio-temporal cube blocks and back.
+// gather raster (t, h, w) tokens into spatio-temporal cube blocks and back,
+// or, in Hilbert order (DFSAttn abstract: Hilbert-curve token reordering),
+// into runs of tokens along a 3-D Hilbert curve through a slot->token table.
 //
 // One CTA moves one cube of one (tensor, b, h): bs rows of d elements, as
 // 16-byte vectors. Cube-order rows are contiguous (bs*d*esize bytes per cube)
@@ -20,6 +22,7 @@ constexpr int kThreads = 256;
 struct ReorderArgs {
   const char* src[3];
   char* dst[3];
+  const int32_t* token_of_slot;  // Hilbert order: token of every slot (-1: padding)
 };
 
 // direction 0: raster -> cube order; 1: cube order -> raster.
@@ -57,12 +60,20 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(KGeom g, ReorderArgs 
     const int idx = threadIdx.x + k * kThreads;
     const int o = idx >> VPR_LOG2;
     const int c = idx & (VPR - 1);
-    uint32_t lt, r2, lh, lw;
-    g.dv_chcw.divmod(static_cast<uint32_t>(o), lt, r2);
-    g.dv_cw.divmod(r2, lh, lw);
-    const int t = t0 + lt, hh = h0 + lh, w = w0 + lw;
-    const bool valid = (t < g.T) && (hh < g.Hh) && (w < g.W);
-    const int64_t n = (static_cast<int64_t>(t) * g.Hh + hh) * g.W + w;
+    bool valid;
+    int64_t n;
+    if (a.token_of_slot != nullptr) {
+      const int32_t tok = __ldg(&a.token_of_slot[j * g.bs + o]);
+      valid = tok >= 0;
+      n = tok;
+    } else {
+      uint32_t lt, r2, lh, lw;
+      g.dv_chcw.divmod(static_cast<uint32_t>(o), lt, r2);
+      g.dv_cw.divmod(r2, lh, lw);
+      const int t = t0 + lt, hh = h0 + lh, w = w0 + lw;
+      valid = (t < g.T) && (hh < g.Hh) && (w < g.W);
+      n = (static_cast<int64_t>(t) * g.Hh + hh) * g.W + w;
+    }
     const int64_t raster = raster_base + n * sN_bytes + c * 16;
     const int64_t packed = packed_base + static_cast<int64_t>(o) * row_bytes + c * 16;
     ok[k] = valid;
@@ -98,9 +109,10 @@ cudaError_t launch_dir(const sba_plan* p, const KGeom& g, const ReorderArgs& a, 
 }  // namespace
 
 cudaError_t launch_reorder(const sba_plan* p, int direction, const void* src[3], void* dst[3],
-                           cudaStream_t st) {
+                           const int32_t* token_of_slot, cudaStream_t st) {
   KGeom g = make_kgeom(p);
   ReorderArgs a{};
+  a.token_of_slot = token_of_slot;
   int n = 0;
   for (int i = 0; i < 3; ++i) {
     if (src[i] == nullptr) continue;

@@ -55,6 +55,7 @@ class Workload:
     rope_split: Optional[tuple] = None  # (t, h, w) widths, sum = d
     per_head_modes: bool = True
     amp_range: Optional[tuple] = None  # (lo, hi) for per-head amplitude scale
+    order: str = "cube"  # block organisation the layer is run with ("cube" / "hilbert")
 
     @property
     def N(self) -> int:
@@ -91,10 +92,16 @@ WORKLOADS = {
 
 
 def custom(name: str, B: int, H: int, T: int, Hh: int, W: int, d: int, cube, dtype="bf16",
-           top_p=(0.9,), top_k=4, rope_split=None, per_head_modes=True, amp_range=None) -> Workload:
+           top_p=(0.9,), top_k=4, rope_split=None, per_head_modes=True, amp_range=None,
+           order="cube") -> Workload:
     """A workload of any shape, built with the same recipe (used for ragged/edge tests)."""
     return Workload(name, B, H, T, Hh, W, d, tuple(cube), dtype, tuple(top_p), top_k,
-                    rope_split, per_head_modes, amp_range)
+                    rope_split, per_head_modes, amp_range, order)
+
+
+def with_order(wl: Workload, order: str) -> Workload:
+    """The same inputs run with another block organisation."""
+    return dataclasses.replace(wl, name=f"{wl.name}_{order}", order=order)
 
 
 def _coords(T: int, Hh: int, W: int):
@@ -201,4 +208,4 @@ def random_qkv(B: int, H: int, N: int, d: int, dtype=torch.bfloat16, seed: int =
     return tuple(out)
 
 
-__all__ = ["Workload", "WORKLOADS", "STRESS_P", "custom", "generate", "random_qkv"]
+__all__ = ["Workload", "WORKLOADS", "STRESS_P", "custom", "generate", "random_qkv", "with_order"]

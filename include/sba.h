@@ -28,6 +28,12 @@
  *   blk*bs + ((t%ct)*ch + h%ch)*cw + w%cw with
  *   blk = ((t/ct)*nH + h/ch)*nW + w/cw (cubes row-major over the cube grid,
  *   tokens row-major inside a cube).
+ * - Hilbert order (DFSAttn: Hilbert-curve token reordering), when the
+ *   geometry's order is SBA_ORDER_HILBERT: a token's slot is its rank along a
+ *   3-D Hilbert curve (Skilling's construction, axes t, h, w) over the
+ *   smallest power-of-two cube holding the grid; each run of bs = ct*ch*cw
+ *   slots is one block, nb = ceil(N/bs), and only the last block has padding
+ *   (slots N .. Npad-1).
  * - Tensors: raster q, k, v, o are [B][H][N][d] with element strides sB, sH,
  *   sN given in the geometry and d contiguous (so [B][N][H][d] storage is
  *   accepted). Reordered qt, kt, vt, ot are packed [B][H][Npad][d].
@@ -72,6 +78,11 @@ typedef enum {
 typedef enum { SBA_F32 = 0, SBA_BF16 = 1 } sba_dtype;
 
 typedef enum {
+  SBA_ORDER_CUBE = 0,       /* blocks are ct x ch x cw cubes of the grid */
+  SBA_ORDER_HILBERT = 1     /* blocks are runs of bs tokens along a 3-D Hilbert curve */
+} sba_order;
+
+typedef enum {
   SBA_SCHED_LPT = 0,        /* persistent CTAs, rows taken longest first */
   SBA_SCHED_HEAD_MAJOR = 1  /* one CTA per row, rows in (b, h, i) order */
 } sba_sched;
@@ -84,6 +95,8 @@ typedef struct {
   int32_t ct, ch, cw;    /* cube extents; bs = ct*ch*cw */
   int32_t dtype;         /* sba_dtype of q, k, v, o and their reordered forms */
   int64_t sB, sH, sN;    /* element strides of raster q/k/v/o; d is contiguous */
+  int32_t order;         /* sba_order; SBA_ORDER_CUBE unless set */
+  int32_t reserved;      /* must be 0 */
 } sba_geometry;
 
 /* Sizes derived from a geometry. */
@@ -111,20 +124,26 @@ SBA_API void sba_plan_destroy(sba_plan* plan);
 SBA_API sba_status sba_plan_query(const sba_plan* plan, sba_plan_info* info);
 
 /* Zero the control words at the start of a workspace (status word and the
- * scheduler's counters). Call once after allocating a workspace, before its
- * first use; a workspace allocated zero-filled needs no call. */
+ * scheduler's counters) and, for Hilbert-order plans, upload the plan's
+ * permutation table into it. Call once after allocating a workspace, before
+ * its first use (required for Hilbert order; for cube order a workspace
+ * allocated zero-filled needs no call). */
 SBA_API sba_status sba_workspace_init(const sba_plan* plan, void* workspace, void* stream);
 
 /* Video-aware block organization (FVAttn abstract): gather raster q, k, v into
- * cube order. Each of the three (src, dst) pairs may be (NULL, NULL) to skip
- * that tensor. Padding slots are written as zeros. Bit copy: no rounding. */
+ * block order. Each of the three (src, dst) pairs may be (NULL, NULL) to skip
+ * that tensor. Padding slots are written as zeros. Bit copy: no rounding.
+ * workspace: may be NULL for cube order; for Hilbert order the workspace
+ * initialised by sba_workspace_init (it holds the permutation table). */
 SBA_API sba_status sba_reorder(const sba_plan* plan,
                        const void* q, const void* k, const void* v,
-                       void* qt, void* kt, void* vt, void* stream);
+                       void* qt, void* kt, void* vt, const void* workspace, void* stream);
 
 /* Inverse of sba_reorder for the output: ot [B][H][Npad][d] -> o, raster with
- * the geometry's strides. Padding slots are dropped. Bit copy. */
-SBA_API sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o, void* stream);
+ * the geometry's strides. Padding slots are dropped. Bit copy. workspace as
+ * for sba_reorder. */
+SBA_API sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o,
+                                 const void* workspace, void* stream);
 
 /* Block scoring and routing (FVAttn abstract: Top-p routing, Top-k safety
  * floor). For every row r = (b, h, i):

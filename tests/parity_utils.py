@@ -25,13 +25,13 @@ TIE_TOL = 1e-6
 
 
 def geom_of(wl) -> Geom:
-    return Geom(wl.T, wl.Hh, wl.W, *wl.cube)
+    return Geom(wl.T, wl.Hh, wl.W, *wl.cube, order=getattr(wl, "order", "cube"))
 
 
 def run_gpu(wl, q, k, v, sched=0, with_trace=False, top_p=None, top_k=None):
     """All four calls on cuda:0; returns a dict of CPU tensors."""
     import block_sparse_attention_sba_b200 as sba
-    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube, order=getattr(wl, "order", "cube"))
     sa = sba.SparseAttention(plan, device=q.device)
     top_p = wl.top_p_per_head() if top_p is None else top_p
     top_k = wl.top_k if top_k is None else top_k

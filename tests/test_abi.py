@@ -72,6 +72,27 @@ def test_host_permutation_matches_oracle(sba, T, Hh, W, cube):
     assert np.array_equal(got, oracle.slot_of_token(oracle.Geom(T, Hh, W, *cube)))
 
 
+@pytest.mark.parametrize("T,Hh,W,cube", [(4, 8, 8, (4, 4, 4)), (5, 9, 7, (2, 4, 8)),
+                                         (21, 30, 52, (2, 8, 8)), (3, 10, 6, (1, 8, 8))])
+def test_host_hilbert_permutation_matches_oracle(sba, T, Hh, W, cube):
+    plan = sba.Plan(1, 1, T, Hh, W, 64, cube, "bf16", order="hilbert")
+    g = oracle.Geom(T, Hh, W, *cube, order="hilbert")
+    assert (plan.info.nb, plan.info.Npad) == (g.nb, g.Npad)
+    got = np.array(sba.sba_perm_export(plan.handle, T * Hh * W))
+    assert np.array_equal(got, oracle.slot_of_token(g))
+
+
+def test_hilbert_reorder_requires_the_workspace(sba):
+    plan = sba.Plan(1, 2, 4, 8, 8, 64, (4, 4, 4), "bf16", order="hilbert")
+    fake = 1 << 20
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_reorder(plan.handle, fake, None, None, fake, None, None, None, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_unreorder(plan.handle, fake, fake, None, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(d=96), -2),                       # untuned head dim
     (dict(cube=(2, 4, 4)), -2),             # block of 32

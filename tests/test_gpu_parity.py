@@ -26,6 +26,13 @@ SMALL = {
                                        top_p=(0.85,), top_k=2, rope_split=(44, 42, 42)),
     "ragged_f32": datagen.custom("ragged_f32", 1, 2, 5, 6, 7, 64, (4, 4, 4), dtype="f32",
                                  top_p=(0.9,), top_k=1),
+    # Hilbert-curve block organisation (ragged tail block, both tile shapes)
+    "hilbert_d128_bs128": datagen.custom("hilbert_d128_bs128", 1, 3, 5, 20, 19, 128, (2, 8, 8),
+                                         top_p=(0.8, 0.9, 0.95), top_k=3, rope_split=(44, 42, 42),
+                                         order="hilbert"),
+    "hilbert_small": datagen.with_order(datagen.WORKLOADS["small"], "hilbert"),
+    "hilbert_f32": datagen.custom("hilbert_f32", 1, 2, 5, 6, 7, 64, (4, 4, 4), dtype="f32",
+                                  top_p=(0.9,), top_k=1, order="hilbert"),
 }
 
 
@@ -150,9 +157,9 @@ def test_topk_floor_and_cap():
 def _attn_with_csr(wl, q, k, v, row_ptr, col_idx, sched=1):
     import block_sparse_attention_sba_b200 as sba
     g = geom_of(wl)
-    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube, order=wl.order)
     sa = sba.SparseAttention(plan, device=q.device)
-    sba.sba_reorder(plan.handle, q, k, v, sa.qt, sa.kt, sa.vt)
+    sba.sba_reorder(plan.handle, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace)
     rp = torch.tensor(row_ptr, dtype=torch.int32, device=q.device)
     ci = torch.tensor(col_idx if len(col_idx) else [0], dtype=torch.int32, device=q.device)
     wo = torch.tensor(oracle.lpt_order(np.diff(row_ptr), g.nb), dtype=torch.int32, device=q.device)
@@ -233,13 +240,14 @@ def test_bounded_wait_gives_up_and_reports_timeout():
 
 # ----------------------------------------------------------------- full size
 
-FULL = ["wan", "hunyuan", "stress"]
+FULL = ["wan", "hunyuan", "stress", "wan_hilbert"]
 
 
 @pytest.fixture(scope="module", params=FULL)
 def full_case(request):
     name = request.param
-    wl = datagen.WORKLOADS[name]
+    wl = (datagen.with_order(datagen.WORKLOADS["wan"], "hilbert") if name == "wan_hilbert"
+          else datagen.WORKLOADS[name])
     q, k, v = datagen.generate(wl, seed=0, device=_cuda())
     gpu = run_gpu(wl, q, k, v, with_trace=True)
     return name, wl, (q, k, v), gpu

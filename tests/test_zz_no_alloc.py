@@ -23,7 +23,7 @@ def _routing(sba, wl, use_noalloc):
     q, k, v = datagen.generate(wl, seed=3, device=dev)
     plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
     sa = sba.SparseAttention(plan, device=dev)
-    sba.sba_reorder(plan.handle, q, k, v, sa.qt, sa.kt, sa.vt)
+    sba.sba_reorder(plan.handle, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace)
     args = (plan.handle, sa.qt, sa.kt, wl.top_p_per_head(), wl.top_k, sa.bitmask, sa.row_cnt,
             sa.row_ptr, sa.col_idx)
     if use_noalloc:
