@@ -369,3 +369,97 @@ def forward(q, k, v, g: Geom, top_p, top_k: int):
     m = build_mask(qt, kt, g, top_p, top_k)
     ot, lse = attention(qt, kt, vt, g, m["row_ptr"], m["col_idx"])
     return unreorder(ot, g), m, lse
+
+
+# ---------------------------------------------------------------------------
+# Stripe masks (Parameterized Stripe Attention for Efficient Video Generation,
+# Approach: a six-parameter mask M(Tw, To, Ts, Sw, So, Ss) of periodic
+# diagonal stripes, from spatio-temporal locality and RoPE-3D periodicity)
+# ---------------------------------------------------------------------------
+#
+# Reading (the page names the parameters but prints no formula): T* act on the
+# temporal offset between the key block and the query block, S* on their
+# spatial offset; w is a stripe's width, o its offset, s its period (0: the
+# stripe occurs once). On the cube grid, with a block's coordinates (tt, th,
+# tw) and its flattened spatial index sp = th*nW + tw,
+#   dt = tt_key - tt_query,   ds = sp_key - sp_query,
+#   x lies in stripe (w, o, s)  <=>  0 <= x - o < w            (s = 0)
+#                                    (x - o) mod s < w          (s > 0)
+#   keep(query block, key block) <=> dt in (Tw, To, Ts) and ds in (Sw, So, Ss).
+# A band of half-width r around the diagonal is (w, o, s) = (2r+1, -r, 0); a
+# band that recurs every nW blocks of the flattened spatial index (the same
+# column one cube row up or down) uses s = nW.
+
+def in_stripe(x, w: int, o: int, s: int):
+    """x (int or int array) lies in the stripe of width w starting at offset o,
+    repeated with period s (s = 0: not repeated)."""
+    x = np.asarray(x, dtype=np.int64)
+    if s == 0:
+        return (x - o >= 0) & (x - o < w)
+    return np.mod(x - o, s) < w  # numpy's mod is non-negative for s > 0
+
+
+def block_coords(g: Geom):
+    """(tt, sp) of every block in cube order: its temporal cube coordinate and
+    its flattened spatial cube index th*nW + tw."""
+    j = np.arange(g.nb, dtype=np.int64)
+    tt = j // (g.nH * g.nW)
+    sp = j % (g.nH * g.nW)
+    return tt, sp
+
+
+def stripe_keep(g: Geom, prm) -> np.ndarray:
+    """[nb, nb] bool keep matrix of one head, rows = query blocks."""
+    Tw, To, Ts, Sw, So, Ss = (int(v) for v in prm)
+    tt, sp = block_coords(g)
+    dt = tt[None, :] - tt[:, None]
+    ds = sp[None, :] - sp[:, None]
+    return in_stripe(dt, Tw, To, Ts) & in_stripe(ds, Sw, So, Ss)
+
+
+def stripe_keep_loops(g: Geom, prm) -> np.ndarray:
+    """Same as stripe_keep with plain loops over the cube grid (small cases)."""
+    Tw, To, Ts, Sw, So, Ss = (int(v) for v in prm)
+
+    def inside(x, w, o, s):
+        return (0 <= x - o < w) if s == 0 else ((x - o) % s < w)
+
+    keep = np.zeros((g.nb, g.nb), dtype=bool)
+    for qt_ in range(g.nT):
+        for qh in range(g.nH):
+            for qw in range(g.nW):
+                i = (qt_ * g.nH + qh) * g.nW + qw
+                for kt_ in range(g.nT):
+                    for kh in range(g.nH):
+                        for kw in range(g.nW):
+                            j = (kt_ * g.nH + kh) * g.nW + kw
+                            dt = kt_ - qt_
+                            ds = (kh * g.nW + kw) - (qh * g.nW + qw)
+                            keep[i, j] = inside(dt, Tw, To, Ts) and inside(ds, Sw, So, Ss)
+    return keep
+
+
+def csr_from_keep(keep_rows: np.ndarray) -> dict:
+    """Bitmask and CSR of a stack of keep rows [R, nb] (same layout as
+    build_mask: bit j%32 of word j//32, col_idx ascending inside a row)."""
+    keep_rows = np.asarray(keep_rows, dtype=bool)
+    R, nb = keep_rows.shape
+    words = -(-nb // 32)
+    bits = np.zeros((R, words * 32), dtype=bool)
+    bits[:, :nb] = keep_rows
+    bitmask = np.packbits(bits, axis=1, bitorder="little").view("<u4").reshape(R, words)
+    row_cnt = keep_rows.sum(axis=1).astype(np.int64)
+    row_ptr = np.zeros(R + 1, dtype=np.int64)
+    row_ptr[1:] = np.cumsum(row_cnt)
+    col_idx = np.nonzero(keep_rows)[1].astype(np.int64)  # row-major: ascending j per row
+    return {"row_cnt": row_cnt, "row_ptr": row_ptr, "col_idx": col_idx, "bitmask": bitmask}
+
+
+def stripe_mask(g: Geom, params, B: int) -> dict:
+    """Stripe mask of every (b, h, query block) row: params[h] = (Tw, To, Ts,
+    Sw, So, Ss) for head h; rows r = (b*H + h)*nb + i as in build_mask."""
+    if g.order != "cube":
+        raise ValueError("stripe masks are defined on the cube grid")
+    per_head = [stripe_keep(g, prm) for prm in params]
+    rows = np.concatenate([per_head[h] for _ in range(B) for h in range(len(params))], axis=0)
+    return csr_from_keep(rows)

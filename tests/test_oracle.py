@@ -455,3 +455,129 @@ def test_hilbert_pooling_and_dense_attention():
     ref = _dense_sdpa(qt, kt, vt, g)
     np.testing.assert_allclose(Ot[:, :, valid], ref[:, :, valid], atol=1e-12)
     _mask_invariants(oracle.build_mask(qt, kt, g, [0.7, 0.9], 2), [0.7, 0.9], 2, g.nb)
+
+
+# ---------------------------------------------------------------------------
+# Stripe masks (Parameterized Stripe Attention for Efficient Video
+# Generation, Approach: M(Tw, To, Ts, Sw, So, Ss)); the reading is stated in
+# the oracle's header of that section.
+# ---------------------------------------------------------------------------
+
+# nT = 4 temporal cubes, one spatial cube
+G_T4 = oracle.Geom(8, 8, 8, 2, 8, 8)
+# one temporal cube, 2 x 3 spatial cubes (flattened spatial index th*3 + tw)
+G_S6 = oracle.Geom(2, 16, 24, 2, 8, 8)
+
+
+def test_stripe_temporal_period_hand_worked():
+    """Every second frame block (w=1, o=0, s=2): catches a dropped modulo or a
+    period applied to the wrong axis."""
+    want = np.array([[1, 0, 1, 0], [0, 1, 0, 1], [1, 0, 1, 0], [0, 1, 0, 1]], dtype=bool)
+    assert np.array_equal(oracle.stripe_keep(G_T4, (1, 0, 2, 1, 0, 0)), want)
+
+
+def test_stripe_spatial_offset_sign_hand_worked():
+    """ds in {-1, 0} (w=2, o=-1): the key block itself and the one just before
+    it in the flattened spatial order. Catches dt/ds taken as query - key."""
+    want = np.array([[1, 0, 0, 0, 0, 0],
+                     [1, 1, 0, 0, 0, 0],
+                     [0, 1, 1, 0, 0, 0],
+                     [0, 0, 1, 1, 0, 0],
+                     [0, 0, 0, 1, 1, 0],
+                     [0, 0, 0, 0, 1, 1]], dtype=bool)
+    assert np.array_equal(oracle.stripe_keep(G_S6, (1, 0, 0, 2, -1, 0)), want)
+
+
+def test_stripe_spatial_period_hand_worked():
+    """ds = 0 mod 3 (s = nW): the same cube column one cube row up or down."""
+    want = np.array([[1, 0, 0, 1, 0, 0],
+                     [0, 1, 0, 0, 1, 0],
+                     [0, 0, 1, 0, 0, 1],
+                     [1, 0, 0, 1, 0, 0],
+                     [0, 1, 0, 0, 1, 0],
+                     [0, 0, 1, 0, 0, 1]], dtype=bool)
+    assert np.array_equal(oracle.stripe_keep(G_S6, (1, 0, 0, 1, 0, 3)), want)
+
+
+SGEOMS = [oracle.Geom(8, 16, 24, 2, 8, 8), oracle.Geom(5, 9, 7, 2, 4, 8),
+          oracle.Geom(21, 30, 52, 2, 8, 8), oracle.Geom(3, 17, 9, 1, 8, 8)]
+
+
+@pytest.mark.parametrize("g", SGEOMS, ids=str)
+def test_stripe_closed_forms(g):
+    nT, nS = g.nT, g.nH * g.nW
+    full = (2 * nT - 1, -(nT - 1), 0, 2 * nS - 1, -(nS - 1), 0)
+    assert oracle.stripe_keep(g, full).all()
+    assert np.array_equal(oracle.stripe_keep(g, (1, 0, 0, 1, 0, 0)), np.eye(g.nb, dtype=bool))
+    assert not oracle.stripe_keep(g, (0, 0, 0, 1, 0, 0)).any()      # zero width
+    assert not oracle.stripe_keep(g, (1, nT, 0, 1, 0, 0)).any()     # offset past the grid
+    # a period no longer than the width covers every offset
+    assert oracle.stripe_keep(g, (3, 5, 3, 4, -7, 2)).all()
+    # temporal band alone: |tt_i - tt_j| <= 1, spatial index equal
+    tt, sp = oracle.block_coords(g)
+    want = (np.abs(tt[:, None] - tt[None, :]) <= 1) & (sp[:, None] == sp[None, :])
+    assert np.array_equal(oracle.stripe_keep(g, (3, -1, 0, 1, 0, 0)), want)
+
+
+@pytest.mark.parametrize("g", SGEOMS[:2] + SGEOMS[3:], ids=str)
+def test_stripe_vectorised_equals_loops(g):
+    rng = np.random.default_rng(11)
+    for _ in range(12):
+        prm = (int(rng.integers(0, 4)), int(rng.integers(-3, 3)), int(rng.integers(0, 4)),
+               int(rng.integers(0, 7)), int(rng.integers(-6, 6)), int(rng.integers(0, 8)))
+        assert np.array_equal(oracle.stripe_keep(g, prm), oracle.stripe_keep_loops(g, prm)), prm
+
+
+@pytest.mark.parametrize("g", SGEOMS, ids=str)
+def test_stripe_invariants(g):
+    tt, sp = oracle.block_coords(g)
+    # a symmetric band is a symmetric relation
+    band = oracle.stripe_keep(g, (3, -1, 0, 5, -2, 0))
+    assert np.array_equal(band, band.T)
+    # keep depends on (dt, ds) only: equal offsets, equal decisions
+    k = oracle.stripe_keep(g, (2, -1, 3, 3, -1, g.nW))
+    dt = tt[None, :] - tt[:, None]
+    ds = sp[None, :] - sp[:, None]
+    for a in np.unique(dt):
+        for c in np.unique(ds):
+            sel = (dt == a) & (ds == c)
+            assert k[sel].all() or not k[sel].any()
+    # block coordinates cover the cube grid in cube order
+    assert np.array_equal(tt * (g.nH * g.nW) + sp, np.arange(g.nb))
+
+
+def test_stripe_csr_layout_matches_build_mask():
+    """The stripe CSR uses build_mask's layout: with every block kept both give
+    the same row_ptr, col_idx and bitmask."""
+    g = oracle.Geom(5, 9, 7, 2, 4, 8)
+    B, H, d = 1, 2, 8
+    rng = np.random.default_rng(3)
+    Qt = oracle.reorder(rng.standard_normal((B, H, g.N, d)), g)
+    Kt = oracle.reorder(rng.standard_normal((B, H, g.N, d)), g)
+    dense = oracle.build_mask(Qt, Kt, g, [1.0, 1.0], 0)
+    nT, nS = g.nT, g.nH * g.nW
+    full = (2 * nT - 1, -(nT - 1), 0, 2 * nS - 1, -(nS - 1), 0)
+    st = oracle.stripe_mask(g, [full, full], B)
+    for key in ("row_cnt", "row_ptr", "col_idx", "bitmask"):
+        assert np.array_equal(np.asarray(st[key]), np.asarray(dense[key])), key
+
+
+def test_stripe_mask_rows_heads_and_csr():
+    g = oracle.Geom(8, 16, 24, 2, 8, 8)
+    params = [(3, -1, 0, 5, -2, 3), (1, 0, 0, 1, 0, 0), (1, 4, 0, 1, 0, 0)]
+    B, H = 2, 3
+    m = oracle.stripe_mask(g, params, B)
+    R = B * H * g.nb
+    assert m["row_ptr"].shape == (R + 1,) and m["row_ptr"][-1] == m["col_idx"].size
+    assert np.array_equal(np.diff(m["row_ptr"]), m["row_cnt"])
+    bits = np.unpackbits(m["bitmask"].view(np.uint8), axis=1, bitorder="little")[:, :g.nb]
+    for b in range(B):
+        for h in range(H):
+            rows = slice((b * H + h) * g.nb, (b * H + h + 1) * g.nb)
+            assert np.array_equal(bits[rows].astype(bool), oracle.stripe_keep(g, params[h]))
+    for r in range(R):
+        c = m["col_idx"][m["row_ptr"][r]:m["row_ptr"][r + 1]]
+        assert np.all(np.diff(c) > 0) and np.array_equal(c, np.nonzero(bits[r])[0])
+    assert (m["row_cnt"][2 * g.nb:3 * g.nb] == 0).all()  # head 2: offset past the grid
+    with pytest.raises(ValueError):
+        oracle.stripe_mask(oracle.Geom(4, 8, 8, 4, 4, 4, order="hilbert"), params[:1], 1)
