@@ -41,7 +41,7 @@ EXPORTED = ["sba_plan_create", "sba_plan_destroy", "sba_plan_query", "sba_worksp
             "sba_reorder", "sba_unreorder", "sba_build_mask", "sba_attention",
             "sba_check_device_status", "sba_debug_timeout_probe", "sba_perm_export",
             "sba_attention_grid_size", "sba_status_string", "sba_last_error",
-            "sba_build_mask_noalloc"]
+            "sba_build_mask_noalloc", "sba_build_stripe_mask"]
 
 
 class sba_geometry(ctypes.Structure):
@@ -50,6 +50,12 @@ class sba_geometry(ctypes.Structure):
                 ("ct", ctypes.c_int32), ("ch", ctypes.c_int32), ("cw", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("sB", ctypes.c_int64), ("sH", ctypes.c_int64),
                 ("sN", ctypes.c_int64), ("order", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class sba_stripe(ctypes.Structure):
+    """One head's stripe-mask parameters (see sba_build_stripe_mask in sba.h)."""
+    _fields_ = [("Tw", ctypes.c_int32), ("To", ctypes.c_int32), ("Ts", ctypes.c_int32),
+                ("Sw", ctypes.c_int32), ("So", ctypes.c_int32), ("Ss", ctypes.c_int32)]
 
 
 class sba_plan_info(ctypes.Structure):
@@ -73,6 +79,7 @@ _sig = {
     "sba_attention": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp],
     "sba_build_mask_noalloc": [_vp, _vp, _vp, ctypes.POINTER(ctypes.c_float), _i32, _vp, _vp, _vp,
                                _vp, _vp, _vp],
+    "sba_build_stripe_mask": [_vp, ctypes.POINTER(sba_stripe), _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "sba_check_device_status": [_vp, _vp, _vp],
     "sba_debug_timeout_probe": [_vp, _vp, ctypes.c_uint64, _vp],
     "sba_perm_export": [_vp, ctypes.POINTER(ctypes.c_int32)],
@@ -169,6 +176,15 @@ def sba_build_mask_noalloc(plan: int, qt, kt, top_p: Sequence[float], top_k: int
     _check(_lib.sba_build_mask_noalloc(plan, _ptr(qt), _ptr(kt), arr, int(top_k), _ptr(bitmask),
                                        _ptr(row_cnt), _ptr(row_ptr), _ptr(col_idx),
                                        _ptr(work_order), _stream(stream)), "sba_build_mask_noalloc")
+
+
+def sba_build_stripe_mask(plan: int, params, bitmask, row_cnt, row_ptr, col_idx, work_order,
+                          workspace, stream=None) -> None:
+    """params: one (Tw, To, Ts, Sw, So, Ss) per head."""
+    arr = (sba_stripe * len(params))(*[sba_stripe(*[int(x) for x in prm]) for prm in params])
+    _check(_lib.sba_build_stripe_mask(plan, arr, _ptr(bitmask), _ptr(row_cnt), _ptr(row_ptr),
+                                      _ptr(col_idx), _ptr(work_order), _ptr(workspace),
+                                      _stream(stream)), "sba_build_stripe_mask")
 
 
 def sba_attention(plan: int, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse=None,
@@ -277,6 +293,24 @@ class SparseAttention:
         sba_reorder(h, q, k, v, self.qt, self.kt, self.vt, self.workspace, stream)
         sba_build_mask(h, self.qt, self.kt, top_p, top_k, self.bitmask, self.row_cnt,
                        self.row_ptr, self.col_idx, self.work_order, self.workspace, stream)
+        sba_attention(h, self.qt, self.kt, self.vt, self.row_ptr, self.col_idx, self.work_order,
+                      self.ot, self.lse, sched, trace, self.workspace, stream)
+        sba_unreorder(h, self.ot, o, self.workspace, stream)
+        return o
+
+    def stripe(self, q, k, v, params, o=None, sched: int = SBA_SCHED_LPT, trace=None,
+               stream=None):
+        """The same path with a stripe mask (one (Tw, To, Ts, Sw, So, Ss) per
+        head, or one for all heads) in place of Top-p routing."""
+        import torch
+        p = self.plan
+        h = p.handle
+        if o is None:
+            o = torch.empty_like(q)
+        params = list(params) if len(params) == p.H else [tuple(params[0])] * p.H
+        sba_reorder(h, q, k, v, self.qt, self.kt, self.vt, self.workspace, stream)
+        sba_build_stripe_mask(h, params, self.bitmask, self.row_cnt, self.row_ptr, self.col_idx,
+                              self.work_order, self.workspace, stream)
         sba_attention(h, self.qt, self.kt, self.vt, self.row_ptr, self.col_idx, self.work_order,
                       self.ot, self.lse, sched, trace, self.workspace, stream)
         sba_unreorder(h, self.ot, o, self.workspace, stream)

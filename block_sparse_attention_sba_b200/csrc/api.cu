@@ -286,6 +286,30 @@ sba_status sba_build_mask(const sba_plan* plan, const void* qt, const void* kt, 
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_build_mask launch");
 }
 
+sba_status sba_build_stripe_mask(const sba_plan* plan, const sba_stripe* params, uint32_t* bitmask,
+                                 int32_t* row_cnt, int32_t* row_ptr, int32_t* col_idx,
+                                 int32_t* work_order, void* workspace, void* stream) {
+  g_err[0] = '\0';
+  if (!plan || !params || !bitmask || !row_cnt || !row_ptr || !col_idx || !work_order || !workspace)
+    return fail(SBA_ERR_INVALID_ARG, "sba_build_stripe_mask: NULL argument");
+  if (!aligned16(workspace)) return fail(SBA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (plan->g.order != SBA_ORDER_CUBE)
+    return fail(SBA_ERR_UNSUPPORTED, "stripe masks are defined on the cube grid (SBA_ORDER_CUBE)");
+  for (int h = 0; h < plan->g.H; ++h) {
+    const sba_stripe& q = params[h];
+    const int32_t v[6] = {q.Tw, q.To, q.Ts, q.Sw, q.So, q.Ss};
+    for (int k = 0; k < 6; ++k)
+      if (v[k] < -32768 || v[k] > 32767)
+        return fail(SBA_ERR_INVALID_ARG, "params[%d] field %d = %d; must lie in [-32768, 32767]", h, k,
+                    v[k]);
+    if (q.Tw < 0 || q.Ts < 0 || q.Sw < 0 || q.Ss < 0)
+      return fail(SBA_ERR_INVALID_ARG, "params[%d]: widths and periods must be >= 0", h);
+  }
+  cudaError_t e = launch_build_stripe_mask(plan, params, bitmask, row_cnt, row_ptr, col_idx,
+                                           work_order, workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_build_stripe_mask launch");
+}
+
 sba_status sba_attention(const sba_plan* plan, const void* qt, const void* kt, const void* vt,
                          const int32_t* row_ptr, const int32_t* col_idx, const int32_t* work_order,
                          void* ot, float* lse, int32_t sched, uint64_t* trace, void* workspace,

@@ -72,6 +72,10 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
                               const float* top_p, int top_k, uint32_t* bitmask, int32_t* row_cnt,
                               int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
                               void* workspace, cudaStream_t st);
+cudaError_t launch_build_stripe_mask(const sba_plan* p, const sba_stripe* params,
+                                     uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
+                                     int32_t* col_idx, int32_t* work_order, void* workspace,
+                                     cudaStream_t st);
 cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, const void* vt,
                              const int32_t* row_ptr, const int32_t* col_idx,
                              const int32_t* work_order, void* ot, float* lse, int sched,

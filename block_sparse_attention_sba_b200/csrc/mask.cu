@@ -437,6 +437,30 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// row_ptr (exclusive scan of row_cnt), work_order and col_idx from bitmask
+// and row_cnt: shared by the Top-p and the stripe masks.
+cudaError_t launch_scan_expand(const sba_plan* p, const uint32_t* bitmask, const int32_t* row_cnt,
+                               int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
+                               uint32_t* status, cudaStream_t st) {
+  const int R = p->info.rows;
+  const int nb = p->info.nb;
+  const int BH = p->g.B * p->g.H;
+  const size_t scan_smem = (static_cast<size_t>(kScanWarps) * (nb + 1) + 2 * static_cast<size_t>(BH)) * sizeof(int);
+  static thread_local int configured_scan = 0;
+  if (scan_smem > 48 * 1024 && configured_scan < static_cast<int>(scan_smem)) {
+    cudaError_t e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(scan_smem));
+    if (e != cudaSuccess) return e;
+    configured_scan = static_cast<int>(scan_smem);
+  }
+  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, nb, BH, row_cnt, row_ptr, work_order,
+                                                        status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  expand_kernel<<<(R + 7) / 8, 256, 0, st>>>(R, nb, bitmask, row_ptr, col_idx);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 static size_t select_smem_bytes(int d, int nkp) {
@@ -485,22 +509,79 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const int R = p->info.rows;
-  const size_t scan_smem = (static_cast<size_t>(kScanWarps) * (g.nb + 1) + 2 * static_cast<size_t>(BH)) * sizeof(int);
-  static thread_local int configured_scan = 0;
-  if (scan_smem > 48 * 1024 && configured_scan < static_cast<int>(scan_smem)) {
-    e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(scan_smem));
-    if (e != cudaSuccess) return e;
-    configured_scan = static_cast<int>(scan_smem);
-  }
-  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, g.nb, BH, row_cnt, row_ptr, work_order,
-                                                        &ctrl->status);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order, &ctrl->status, st);
+}
 
-  expand_kernel<<<(R + 7) / 8, 256, 0, st>>>(R, g.nb, bitmask, row_ptr, col_idx);
-  return cudaGetLastError();
+// ------------------------------------------------------------ stripe masks
+// Parameterized Stripe Attention for Efficient Video Generation (Approach):
+// M(Tw, To, Ts, Sw, So, Ss). One warp per (head, query block) row writes the
+// row's bitmask words with ballots and its count; the CSR and the work order
+// come from the same scan and expand launches as the Top-p mask.
+namespace {
+
+struct StripeArgs {
+  int16_t p[256][6];  // Tw, To, Ts, Sw, So, Ss per head
+};
+
+__device__ __forceinline__ bool in_stripe(int x, int w, int o, int s) {
+  const int y = x - o;
+  if (s == 0) return y >= 0 && y < w;
+  int m = y % s;
+  if (m < 0) m += s;
+  return m < w;
+}
+
+// grid (ceil(nb / 8), B*H), 256 threads: warp w handles query block
+// blockIdx.x*8 + w of head blockIdx.y.
+__global__ void __launch_bounds__(256)
+    stripe_kernel(KGeom g, StripeArgs sa, uint32_t* __restrict__ bitmask,
+                  int32_t* __restrict__ row_cnt) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + warp;
+  if (i >= g.nb) return;  // whole warp
+  const int bh = blockIdx.y;
+  uint32_t b, h;
+  g.dv_H.divmod(static_cast<uint32_t>(bh), b, h);
+  const int Tw = sa.p[h][0], To = sa.p[h][1], Ts = sa.p[h][2];
+  const int Sw = sa.p[h][3], So = sa.p[h][4], Ss = sa.p[h][5];
+  const int nS = g.nH * g.nW;
+  const int qt = i / nS, qs = i - qt * nS;
+  const int words = (g.nb + 31) >> 5;
+  const int64_t r = static_cast<int64_t>(bh) * g.nb + i;
+  int cnt = 0;
+  for (int c = 0; c < words; ++c) {
+    const int j = c * 32 + lane;
+    bool keep = false;
+    if (j < g.nb) {
+      const int kt = j / nS, ks = j - kt * nS;
+      keep = in_stripe(kt - qt, Tw, To, Ts) && in_stripe(ks - qs, Sw, So, Ss);
+    }
+    const uint32_t word = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) bitmask[r * words + c] = word;
+    cnt += __popc(word);
+  }
+  if (lane == 0) row_cnt[r] = cnt;
+}
+
+}  // namespace
+
+cudaError_t launch_build_stripe_mask(const sba_plan* p, const sba_stripe* params,
+                                     uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
+                                     int32_t* col_idx, int32_t* work_order, void* workspace,
+                                     cudaStream_t st) {
+  KGeom g = make_kgeom(p);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(static_cast<char*>(workspace) + p->ws_ctrl);
+  StripeArgs sa;
+  for (int h = 0; h < 256; ++h) {
+    const sba_stripe q = h < g.H ? params[h] : sba_stripe{0, 0, 0, 0, 0, 0};
+    const int32_t v[6] = {q.Tw, q.To, q.Ts, q.Sw, q.So, q.Ss};
+    for (int k = 0; k < 6; ++k) sa.p[h][k] = static_cast<int16_t>(v[k]);
+  }
+  dim3 grid((g.nb + 7) / 8, g.B * g.H);
+  stripe_kernel<<<grid, 256, 0, st>>>(g, sa, bitmask, row_cnt);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order, &ctrl->status, st);
 }
 
 // ------------------------------------------------------------------------

@@ -12,6 +12,8 @@
  *   sba_reorder     raster (t,h,w) tokens -> spatio-temporal cube blocks
  *   sba_build_mask  pooled block scores -> Top-p / Top-k mask (bitmask + CSR)
  *                   and a longest-first work order
+ *                   (sba_build_stripe_mask: the same outputs from a static
+ *                   stripe pattern instead of scores)
  *   sba_attention   online-softmax attention over the selected key blocks
  *   sba_unreorder   cube blocks -> raster tokens
  *
@@ -113,6 +115,12 @@ typedef struct {
 
 typedef struct sba_plan sba_plan;
 
+/* Parameters of one head's stripe mask (sba_build_stripe_mask). */
+typedef struct {
+  int32_t Tw, To, Ts; /* temporal stripe: width, offset, period (0: once) */
+  int32_t Sw, So, Ss; /* spatial stripe: width, offset, period (0: once) */
+} sba_stripe;
+
 /* Validate a geometry and build a host-side plan (no device memory, no CUDA
  * call). Supported: bs in {64, 128}; bf16 with d in {64, 128}; f32 with d = 64;
  * nb <= 1024; B*H <= 8192; H <= 256; R*nb < 2^31; strides multiples of 8
@@ -194,6 +202,33 @@ SBA_API sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* qt, 
                                           const float* top_p, int32_t top_k,
                                           uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
                                           int32_t* col_idx, int32_t* work_order, void* stream);
+
+/* Stripe mask (Parameterized Stripe Attention for Efficient Video Generation,
+ * Approach: a six-parameter mask M(Tw, To, Ts, Sw, So, Ss) of periodic
+ * diagonal stripes). A static alternative to sba_build_mask that needs no
+ * scores: rows, outputs and their layout are those of sba_build_mask, and
+ * sba_attention consumes them unchanged. The page names the parameters but
+ * prints no formula; this library reads them as follows. A block has cube
+ * coordinates (tt, th, tw) and flattened spatial index sp = th*nW + tw; for
+ * query block i and key block j
+ *   dt = tt_j - tt_i,   ds = sp_j - sp_i,
+ *   x lies in stripe (w, o, s) when 0 <= x - o < w (s == 0), or when
+ *   ((x - o) mod s) < w with the non-negative remainder (s > 0);
+ *   block j is kept for row i when dt lies in (Tw, To, Ts) and ds in
+ *   (Sw, So, Ss) of the row's head.
+ * A band of half-width r around the diagonal is (2r+1, -r, 0); s = nW
+ * repeats a spatial stripe every cube row. Rows may come out empty (their
+ * attention output is zero, lse -inf).
+ * params: host array [H], one per head; every width and period >= 0 and
+ * every field within [-32768, 32767], else SBA_ERR_INVALID_ARG. Cube order
+ * only: plans with SBA_ORDER_HILBERT return SBA_ERR_UNSUPPORTED. Outputs
+ * (device, caller-owned) as for sba_build_mask; workspace as for
+ * sba_build_mask (its control block records device-side check failures).
+ * Integer work only: results are exact. */
+SBA_API sba_status sba_build_stripe_mask(const sba_plan* plan, const sba_stripe* params,
+                                         uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
+                                         int32_t* col_idx, int32_t* work_order, void* workspace,
+                                         void* stream);
 
 /* Block-sparse attention forward (FVAttn abstract: attention over the
  * materialised mask). For every real query slot q of block i:

@@ -153,3 +153,31 @@ def test_binding_has_no_fallback_path():
     src = open(os.path.join(ROOT, "block_sparse_attention_sba_b200", "__init__.py")).read()
     assert "oracle" not in src.replace("no fallback", "")
     assert "numpy" not in src and "scaled_dot_product" not in src
+
+
+def test_stripe_mask_validates_before_any_launch(sba):
+    plan = sba.Plan(1, 2, 4, 8, 8, 64, (4, 4, 4), "bf16")
+    h = plan.handle
+    fake = 1 << 20  # never dereferenced: validation fails first
+    ok = (3, -1, 0, 5, -2, 0)
+    for bad in [(-1, 0, 0, 1, 0, 0), (1, 0, -2, 1, 0, 0), (1, 0, 0, -3, 0, 0), (1, 0, 0, 1, 0, -1),
+                (1, 40000, 0, 1, 0, 0), (1, 0, 0, 1, -40000, 0)]:
+        with pytest.raises(sba.SbaError) as e:
+            sba.sba_build_stripe_mask(h, [ok, bad], fake, fake, fake, fake, fake, fake, stream=0)
+        assert e.value.status == sba.SBA_ERR_INVALID_ARG, bad
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_build_stripe_mask(h, [ok, ok], fake, fake, fake, fake, fake, fake + 8, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG  # misaligned workspace
+    hplan = sba.Plan(1, 2, 4, 8, 8, 64, (4, 4, 4), "bf16", order="hilbert")
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_build_stripe_mask(hplan.handle, [ok, ok], fake, fake, fake, fake, fake, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_UNSUPPORTED
+    assert "cube" in sba.sba_last_error()
+
+
+def test_stripe_struct_matches_the_header(sba):
+    import ctypes
+    assert ctypes.sizeof(sba.sba_stripe) == 24
+    text = open(os.path.join(ROOT, "include", "sba.h")).read()
+    assert "int32_t Tw, To, Ts;" in text and "int32_t Sw, So, Ss;" in text
+    assert [f[0] for f in sba.sba_stripe._fields_] == ["Tw", "To", "Ts", "Sw", "So", "Ss"]
