@@ -463,3 +463,179 @@ def stripe_mask(g: Geom, params, B: int) -> dict:
     per_head = [stripe_keep(g, prm) for prm in params]
     rows = np.concatenate([per_head[h] for _ in range(B) for h in range(len(params))], axis=0)
     return csr_from_keep(rows)
+
+
+# ---------------------------------------------------------------------------
+# Low-bit P.V (VC-Attention: Value Smoothing and Softmax Casting for Low-bit
+# Attention, abstract: V-Smooth and ExpCast-FP8)
+# ---------------------------------------------------------------------------
+#
+# Readings (the abstract gives the ideas, not the formulas):
+# * E4M3 is the "fn" encoding: sign bit 7, exponent bits 3..6 with bias 7,
+#   mantissa bits 0..2, exponent 0 subnormal (M/8 * 2^-6), code 0x7F NaN, no
+#   infinities, largest finite 448. Encoding rounds to nearest, ties to the
+#   even code, and saturates at +-448.
+# * V-Smooth: for every key block j, mu_j = mean of V over the block's real
+#   tokens; the residual R = V - mu_j (zero on padding slots) is quantised to
+#   E4M3 with one power-of-two scale per (batch, head), sigma = 2^e with e the
+#   smallest integer such that max|R| <= 448 * 2^e (e = 0 when R is all zero),
+#   so that one fp32 accumulator serves every block. The mean comes back
+#   through the per-block row sums: sum_j l_j mu_j with l_j the sum of the
+#   block's probabilities. mu_j, R and the scaling are evaluated in fp32 (the
+#   kernels' precision), the quantisation decision on the fp32 values. The
+#   page's online clustering of value tokens is not built: cube blocks already
+#   hold spatio-temporal neighbours.
+# * ExpCast-FP8: the probability code of a log2-domain score x taken relative
+#   to the row's reference maximum (x <= 0 at the reference) is
+#   c = clamp(rint(8x + 120), 0, 126): one multiply-add puts the integer part
+#   of x + 15 into the exponent field and eighths of its fraction into the
+#   mantissa field, so decode(c) interpolates 2^(x+8) linearly between powers
+#   of two (exact where 8x is an integer and -14 <= x <= 0). The reference
+#   maps to 2^8 rather than 1 so that normal codes cover 14 octaves below the
+#   maximum; the factor cancels in the normalisation and lse removes it.
+# * Reference maximum: the row maximum of the first selected block; a later
+#   block whose maximum exceeds the reference by more than 0.75 (log2 units)
+#   replaces it (the accumulators are rescaled by 2^(old - new)), so that no
+#   code exceeds 126. With low-bit codes the reference changes the result, so
+#   this rule is part of the definition.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(code) -> np.ndarray:
+    """Values of E4M3 codes (0..255)."""
+    c = np.asarray(code, dtype=np.int64)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return np.where(c & 0x80, -mag, mag)
+
+
+_E4M3_POS = e4m3_decode(np.arange(127))  # finite non-negative values, codes 0..126, ascending
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest E4M3 code of x (ties to the even code), saturating at +-448."""
+    x = np.asarray(x, dtype=np.float64)
+    ax = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3_POS, ax), 1, 126)
+    lo = hi - 1
+    dlo = ax - _E4M3_POS[lo]
+    dhi = _E4M3_POS[hi] - ax
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(ax >= _E4M3_POS[126], 126, code)
+    sign = (x < 0) & (code > 0)
+    return (code | np.where(sign, 0x80, 0)).astype(np.uint8)
+
+
+EXPCAST_BIAS = 120.0  # code of the reference maximum (value 2^8)
+EXPCAST_TAU = 0.75    # reference replacement threshold, log2 units
+
+
+def expcast_code(x) -> np.ndarray:
+    """ExpCast-FP8 probability code of log2-domain scores x relative to the
+    reference maximum (reading above)."""
+    y = np.rint(8.0 * np.asarray(x, dtype=np.float64) + EXPCAST_BIAS)
+    return np.clip(np.nan_to_num(y, nan=0.0, neginf=0.0), 0, 126).astype(np.int64)
+
+
+def v_smooth(Vt: np.ndarray, g: Geom):
+    """V-Smooth quantisation of cube-ordered values Vt [B,H,Npad,d].
+
+    Returns (codes uint8 [B,H,Npad,d], mu fp32 [B,H,nb,d], e int [B,H])."""
+    B, H, Npad, d = Vt.shape
+    nb, bs = g.nb, g.bs
+    valid = slot_valid(g)
+    V32 = np.asarray(Vt, dtype=np.float32).reshape(B, H, nb, bs, d)
+    vmask = valid.reshape(nb, bs)[None, None, :, :, None]
+    cnt = valid.reshape(nb, bs).sum(axis=1).astype(np.float64)[None, None, :, None]
+    mu = (np.where(vmask, V32.astype(np.float64), 0.0).sum(axis=3) / cnt).astype(np.float32)
+    R = np.where(vmask, V32 - mu[:, :, :, None, :], np.float32(0.0)).astype(np.float32)
+    e = np.zeros((B, H), dtype=np.int64)
+    codes = np.zeros((B, H, nb, bs, d), dtype=np.uint8)
+    for b in range(B):
+        for h in range(H):
+            amax = float(np.abs(R[b, h]).max())
+            if amax > 0.0:
+                k = int(math.ceil(math.log2(amax / E4M3_MAX)))
+                while amax > E4M3_MAX * 2.0 ** k:  # guard the log2 rounding
+                    k += 1
+                while k > -149 and amax <= E4M3_MAX * 2.0 ** (k - 1):
+                    k -= 1
+                e[b, h] = k
+            scaled = (R[b, h] * np.float32(2.0 ** -int(e[b, h]))).astype(np.float32)
+            codes[b, h] = e4m3_encode(scaled)
+    return codes.reshape(B, H, Npad, d), mu, e
+
+
+def v_smooth_dequant(codes: np.ndarray, mu: np.ndarray, e: np.ndarray, g: Geom) -> np.ndarray:
+    """sigma * decode(codes) + mu_j on real slots, 0 on padding: the values the
+    low-bit path effectively attends to."""
+    B, H, Npad, d = codes.shape
+    valid = slot_valid(g)
+    R = e4m3_decode(codes) * np.exp2(e.astype(np.float64))[:, :, None, None]
+    Vd = R + np.repeat(mu.astype(np.float64), g.bs, axis=2)
+    return np.where(valid[None, None, :, None], Vd, 0.0)
+
+
+def attention_fp8(Qt, Kt, codes, mu, e, g: Geom, row_ptr, col_idx, blocks=None):
+    """Block-sparse attention with ExpCast-FP8 probabilities and V-Smooth
+    values (readings above), row by row in col_idx order.
+
+    Per selected block j of a row, on its real keys: x = q.k / sqrt(d) * log2(e)
+    - m, probabilities P = decode(expcast_code(x)), l_j = sum of P over the
+    block; accumulators A += P @ (sigma * decode(codes_j)), L += l_j,
+    M += l_j * mu_j, all rescaled together when the reference m changes.
+    O = (A + M) / L, lse = ln(L) + (m - 8) * ln(2). Padding query slots:
+    O = 0, lse = 0. Returns (Ot, lse) like ``attention``."""
+    Qt = np.asarray(Qt, dtype=np.float64)
+    Kt = np.asarray(Kt, dtype=np.float64)
+    B, H, Npad, d = Qt.shape
+    nb, bs = g.nb, g.bs
+    valid = slot_valid(g)
+    Vr = e4m3_decode(codes) * np.exp2(np.asarray(e, dtype=np.float64))[:, :, None, None]
+    Ot = np.full((B, H, Npad, d), np.nan)
+    lse = np.full((B, H, Npad), np.nan)
+    if blocks is None:
+        blocks = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
+    c2 = math.log2(math.e) / math.sqrt(d)
+    for (b, h, i) in blocks:
+        r = (b * H + h) * nb + i
+        sel = np.asarray(col_idx[row_ptr[r]:row_ptr[r + 1]], dtype=np.int64)
+        q_slots = np.arange(i * bs, (i + 1) * bs)
+        q = Qt[b, h, q_slots]
+        n_q = q.shape[0]
+        m = np.full(n_q, -np.inf)
+        A = np.zeros((n_q, d))
+        L = np.zeros(n_q)
+        M = np.zeros((n_q, d))
+        for idx, j in enumerate(sel):
+            ks = np.arange(j * bs, (j + 1) * bs)
+            ks = ks[valid[ks]]
+            x = (q @ Kt[b, h, ks].T) * c2
+            mblk = x.max(axis=1)
+            if idx == 0:
+                m_new = mblk
+            else:
+                m_new = np.where(mblk > m + EXPCAST_TAU, mblk, m)
+            alpha = np.where(np.isfinite(m), np.exp2(np.where(np.isfinite(m), m - m_new, 0.0)), 0.0)
+            A *= alpha[:, None]
+            M *= alpha[:, None]
+            L *= alpha
+            m = m_new
+            P = e4m3_decode(expcast_code(x - m[:, None]))
+            lj = P.sum(axis=1)
+            A += P @ Vr[b, h, ks]
+            M += lj[:, None] * mu[b, h, j].astype(np.float64)[None, :]
+            L += lj
+        qv = valid[q_slots]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            o = (A + M) / L[:, None]
+            ls = np.log(L) + (m - 8.0) * math.log(2.0)
+        o[~qv] = 0.0
+        ls[~qv] = 0.0
+        Ot[b, h, q_slots] = o
+        lse[b, h, q_slots] = ls
+    return Ot, lse

@@ -581,3 +581,175 @@ def test_stripe_mask_rows_heads_and_csr():
     assert (m["row_cnt"][2 * g.nb:3 * g.nb] == 0).all()  # head 2: offset past the grid
     with pytest.raises(ValueError):
         oracle.stripe_mask(oracle.Geom(4, 8, 8, 4, 4, 4, order="hilbert"), params[:1], 1)
+
+
+# ---------------------------------------------------------------------------
+# Low-bit P.V (VC-Attention abstract: V-Smooth, ExpCast-FP8); the readings
+# are stated in the oracle's header of that section.
+# ---------------------------------------------------------------------------
+from oracle import oracle as _o  # noqa: E402
+
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    torch = pytest.importorskip("torch")
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = _o.e4m3_decode(np.arange(256))
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+    assert got[126] == 448.0 and got[1] == 2.0 ** -9 and got[8] == 2.0 ** -6 and got[56] == 1.0
+
+
+def test_e4m3_encode_matches_torch_in_range_and_saturates():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.uniform(-4, 2.6, 20000),
+                        _o.e4m3_decode(np.arange(127)), -_o.e4m3_decode(np.arange(1, 127))])
+    x = x[np.abs(x) <= 448.0].astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = _o.e4m3_encode(x)
+    # torch writes -0 for negatives that round to zero; compare values there
+    same = (got == ref) | ((_o.e4m3_decode(got) == 0) & (_o.e4m3_decode(ref) == 0))
+    assert same.all()
+    assert _o.e4m3_encode([500.0, 1e9, -449.0])[:].tolist() == [126, 126, 254]
+    # ties go to the even code: 1.0625 lies between 1.0 (56) and 1.125 (57)
+    assert _o.e4m3_encode([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10]).tolist() == [56, 58, 0, 2]
+
+
+def test_expcast_code_closed_forms():
+    k = np.arange(-14, 1)
+    assert np.array_equal(_o.e4m3_decode(_o.expcast_code(k)), np.exp2(k + 8.0))
+    assert _o.expcast_code([0.0, 0.75, -np.inf, np.nan, -50.0, 1.0, 100.0]).tolist() == \
+        [120, 126, 0, 0, 0, 126, 126]
+    x = np.linspace(-14, 0.75, 20001)
+    c = _o.expcast_code(x)
+    assert np.all(np.diff(c) >= 0)                      # monotone
+    rel = _o.e4m3_decode(c) / np.exp2(x + 8.0) - 1.0
+    # piecewise-linear 2^x (at most +8.61 % at fraction 1/ln2 - 1) and rounding
+    # to eighths (a factor 2^(+-1/16)) bound the relative error
+    assert rel.max() <= (1 + 0.0861) * 2 ** (1 / 16) - 1 + 1e-9
+    assert rel.min() >= 2 ** (-1 / 16) - 1 - 1e-9
+
+
+def _vsmooth_case(seed=0, g=oracle.Geom(5, 9, 7, 2, 4, 8)):
+    rng = np.random.default_rng(seed)
+    B, H, d = 1, 2, 16
+    Vt = oracle.reorder(rng.standard_normal((B, H, g.N, d)) * 3.0 + rng.standard_normal(d), g)
+    return g, Vt
+
+
+def test_v_smooth_error_bound_scale_and_means():
+    g, Vt = _vsmooth_case()
+    codes, mu, e = _o.v_smooth(Vt, g)
+    valid = oracle.slot_valid(g)
+    # mu_j is the plain average over the block's real tokens (slot loop)
+    for j in range(g.nb):
+        sl = [s for s in range(j * g.bs, (j + 1) * g.bs) if valid[s]]
+        assert np.allclose(mu[0, 1, j], Vt[0, 1, sl].mean(axis=0), rtol=1e-6, atol=1e-6)
+    R = np.where(valid[None, None, :, None], Vt - np.repeat(mu, g.bs, axis=2), 0.0)
+    sig = np.exp2(e.astype(float))[:, :, None, None]
+    amax = np.abs(R).max(axis=(2, 3))
+    assert np.all(amax <= 448.0 * np.exp2(e)) and np.all(amax > 224.0 * np.exp2(e))
+    deq = _o.e4m3_decode(codes) * sig
+    assert np.all(np.abs(deq - R) <= np.maximum(2.0 ** -4 * np.abs(R), 2.0 ** -10 * sig) + 1e-6)
+    assert np.all(codes[0, :, ~valid] == 0)
+    assert np.allclose(_o.v_smooth_dequant(codes, mu, e, g), np.where(valid[None, None, :, None],
+                       deq + np.repeat(mu, g.bs, axis=2), 0.0))
+
+
+def test_v_smooth_is_exact_on_block_constant_values():
+    g = oracle.Geom(5, 9, 7, 2, 4, 8)
+    rng = np.random.default_rng(2)
+    per_block = rng.standard_normal((1, 1, g.nb, 8)).astype(np.float32)
+    Vt = np.repeat(per_block, g.bs, axis=2) * oracle.slot_valid(g)[None, None, :, None]
+    codes, mu, e = _o.v_smooth(Vt, g)
+    assert not codes.any() and e[0, 0] == 0
+    assert np.array_equal(mu, per_block)
+
+
+def _fp8_attention_case(seed=1, scale_v=1.0, shift_v=0.0):
+    g = oracle.Geom(5, 9, 7, 2, 4, 8)
+    rng = np.random.default_rng(seed)
+    B, H, d = 1, 2, 16
+    Qt = oracle.reorder(rng.standard_normal((B, H, g.N, d)) * 2.0, g)
+    Kt = oracle.reorder(rng.standard_normal((B, H, g.N, d)), g)
+    Vt = oracle.reorder(rng.standard_normal((B, H, g.N, d)) * scale_v + shift_v, g)
+    R = B * H * g.nb
+    sel = [np.sort(rng.choice(g.nb, size=int(rng.integers(1, g.nb + 1)), replace=False))
+           for _ in range(R)]
+    row_ptr = np.concatenate([[0], np.cumsum([s.size for s in sel])])
+    col_idx = np.concatenate(sel)
+    return g, Qt, Kt, Vt, row_ptr, col_idx
+
+
+def test_fp8_attention_is_close_to_exact_attention():
+    g, Qt, Kt, Vt, rp, ci = _fp8_attention_case()
+    codes, mu, e = _o.v_smooth(Vt, g)
+    O8, l8 = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci)
+    O, l = oracle.attention(Qt, Kt, Vt, g, rp, ci)
+    v = oracle.slot_valid(g)
+    rel = np.linalg.norm(O8[:, :, v] - O[:, :, v]) / np.linalg.norm(O[:, :, v])
+    assert rel < 0.05, rel
+    # the probability codes err by at most ~+12 %/-4.3 % where they matter, so
+    # the log of the denominator moves by little
+    assert np.abs(l8[:, :, v] - l[:, :, v]).max() < math.log(1.12)
+
+
+def test_fp8_attention_rows_are_convex_combinations_of_the_dequantised_values():
+    g, Qt, Kt, Vt, rp, ci = _fp8_attention_case(seed=4)
+    codes, mu, e = _o.v_smooth(Vt, g)
+    O8, _ = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci)
+    Vd = _o.v_smooth_dequant(codes, mu, e, g)
+    v = oracle.slot_valid(g)
+    B, H = Qt.shape[:2]
+    for b in range(B):
+        for h in range(H):
+            for i in range(g.nb):
+                r = (b * H + h) * g.nb + i
+                keys = np.concatenate([np.arange(j * g.bs, (j + 1) * g.bs) for j in ci[rp[r]:rp[r + 1]]])
+                keys = keys[v[keys]]
+                o = O8[b, h, i * g.bs:(i + 1) * g.bs][v[i * g.bs:(i + 1) * g.bs]]
+                assert np.all(o <= Vd[b, h, keys].max(axis=0) + 1e-9)
+                assert np.all(o >= Vd[b, h, keys].min(axis=0) - 1e-9)
+
+
+def test_fp8_attention_power_of_two_and_shift_equivariance():
+    """Scaling V by 2 only moves the per-head exponent (same codes, O doubles
+    exactly); adding one vector to every value moves only the block means (O
+    moves by that vector): catches a dropped scale or a dropped mean term."""
+    g, Qt, Kt, Vt, rp, ci = _fp8_attention_case(seed=3)
+    v = oracle.slot_valid(g)
+    c1, m1, e1 = _o.v_smooth(Vt, g)
+    O1, _ = _o.attention_fp8(Qt, Kt, c1, m1, e1, g, rp, ci)
+    c2, m2, e2 = _o.v_smooth(Vt * 2.0, g)
+    assert np.array_equal(c1, c2) and np.array_equal(e2, e1 + 1)
+    O2, _ = _o.attention_fp8(Qt, Kt, c2, m2, e2, g, rp, ci)
+    assert np.array_equal(O2, 2.0 * O1)
+    shift = np.array([0.5, -1.25] + [0.0] * 14)
+    Vs = np.where(v[None, None, :, None], Vt + shift, 0.0)
+    c3, m3, e3 = _o.v_smooth(Vs, g)
+    O3, _ = _o.attention_fp8(Qt, Kt, c3, m3, e3, g, rp, ci)
+    assert np.allclose(O3[:, :, v], O1[:, :, v] + shift, atol=1e-5)
+
+
+def test_fp8_reference_max_is_replaced_when_a_later_block_dominates():
+    """A row whose second block scores 20 (log2 units) above its first: the
+    first block's weight falls to 0 and the output is the second block's own
+    low-bit average. Without replacing the reference the codes would clip at
+    448 and the output would move."""
+    g = oracle.Geom(4, 8, 8, 4, 4, 4)  # nb = 4 full blocks of 64
+    rng = np.random.default_rng(7)
+    d = 8
+    Qt = np.zeros((1, 1, g.Npad, d)); Qt[..., 0] = 1.0
+    Kt = rng.standard_normal((1, 1, g.Npad, d)) * 0.1
+    boost = 20.0 * math.sqrt(d) / math.log2(math.e)
+    Kt[0, 0, 2 * g.bs:3 * g.bs, 0] += boost
+    Vt = rng.standard_normal((1, 1, g.Npad, d))
+    codes, mu, e = _o.v_smooth(Vt, g)
+    R = g.nb
+    rp = np.arange(R + 1) * 2
+    ci = np.tile([0, 2], R)
+    O8, _ = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci, blocks=[(0, 0, 0)])
+    only2, _ = _o.attention_fp8(Qt, Kt, codes, mu, e, g, np.arange(R + 1), np.full(R, 2),
+                                blocks=[(0, 0, 0)])
+    sl = slice(0, g.bs)
+    assert np.allclose(O8[0, 0, sl], only2[0, 0, sl], atol=1e-4)
