@@ -474,7 +474,8 @@ def stripe_mask(g: Geom, params, B: int) -> dict:
 # * E4M3 is the "fn" encoding: sign bit 7, exponent bits 3..6 with bias 7,
 #   mantissa bits 0..2, exponent 0 subnormal (M/8 * 2^-6), code 0x7F NaN, no
 #   infinities, largest finite 448. Encoding rounds to nearest, ties to the
-#   even code, and saturates at +-448.
+#   even code, saturates at +-448, and keeps the sign of a negative value
+#   that rounds to zero (code 0x80).
 # * V-Smooth: for every key block j, mu_j = mean of V over the block's real
 #   tokens; the residual R = V - mu_j (zero on padding slots) is quantised to
 #   E4M3 with one power-of-two scale per (batch, head), sigma = 2^e with e the
@@ -526,8 +527,8 @@ def e4m3_encode(x) -> np.ndarray:
     pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
     code = np.where(pick_hi, hi, lo)
     code = np.where(ax >= _E4M3_POS[126], 126, code)
-    sign = (x < 0) & (code > 0)
-    return (code | np.where(sign, 0x80, 0)).astype(np.uint8)
+    # a negative value keeps its sign bit even when it rounds to zero (-0)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
 
 
 EXPCAST_BIAS = 120.0  # code of the reference maximum (value 2^8)
