@@ -41,7 +41,8 @@ EXPORTED = ["sba_plan_create", "sba_plan_destroy", "sba_plan_query", "sba_worksp
             "sba_reorder", "sba_unreorder", "sba_build_mask", "sba_attention",
             "sba_check_device_status", "sba_debug_timeout_probe", "sba_perm_export",
             "sba_attention_grid_size", "sba_status_string", "sba_last_error",
-            "sba_build_mask_noalloc", "sba_build_stripe_mask"]
+            "sba_build_mask_noalloc", "sba_build_stripe_mask", "sba_smooth_v",
+            "sba_lowbit_scratch_bytes", "sba_attention_lowbit"]
 
 
 class sba_geometry(ctypes.Structure):
@@ -80,6 +81,10 @@ _sig = {
     "sba_build_mask_noalloc": [_vp, _vp, _vp, ctypes.POINTER(ctypes.c_float), _i32, _vp, _vp, _vp,
                                _vp, _vp, _vp],
     "sba_build_stripe_mask": [_vp, ctypes.POINTER(sba_stripe), _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "sba_smooth_v": [_vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "sba_lowbit_scratch_bytes": [_vp, ctypes.POINTER(ctypes.c_size_t)],
+    "sba_attention_lowbit": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                             ctypes.c_size_t, _vp, _vp],
     "sba_check_device_status": [_vp, _vp, _vp],
     "sba_debug_timeout_probe": [_vp, _vp, ctypes.c_uint64, _vp],
     "sba_perm_export": [_vp, ctypes.POINTER(ctypes.c_int32)],
@@ -185,6 +190,26 @@ def sba_build_stripe_mask(plan: int, params, bitmask, row_cnt, row_ptr, col_idx,
     _check(_lib.sba_build_stripe_mask(plan, arr, _ptr(bitmask), _ptr(row_cnt), _ptr(row_ptr),
                                       _ptr(col_idx), _ptr(work_order), _ptr(workspace),
                                       _stream(stream)), "sba_build_stripe_mask")
+
+
+def sba_smooth_v(plan: int, vt, vq, vmean, vexp, workspace, stream=None) -> None:
+    _check(_lib.sba_smooth_v(plan, _ptr(vt), _ptr(vq), _ptr(vmean), _ptr(vexp), _ptr(workspace),
+                             _stream(stream)), "sba_smooth_v")
+
+
+def sba_lowbit_scratch_bytes(plan: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.sba_lowbit_scratch_bytes(plan, ctypes.byref(out)), "sba_lowbit_scratch_bytes")
+    return int(out.value)
+
+
+def sba_attention_lowbit(plan: int, qt, kt, vq, vmean, vexp, row_ptr, col_idx, work_order, ot,
+                         lse=None, trace=None, scratch=None, scratch_bytes: int = 0,
+                         workspace=None, stream=None) -> None:
+    _check(_lib.sba_attention_lowbit(plan, _ptr(qt), _ptr(kt), _ptr(vq), _ptr(vmean), _ptr(vexp),
+                                     _ptr(row_ptr), _ptr(col_idx), _ptr(work_order), _ptr(ot),
+                                     _ptr(lse), _ptr(trace), _ptr(scratch), int(scratch_bytes),
+                                     _ptr(workspace), _stream(stream)), "sba_attention_lowbit")
 
 
 def sba_attention(plan: int, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse=None,
@@ -313,6 +338,34 @@ class SparseAttention:
                               self.work_order, self.workspace, stream)
         sba_attention(h, self.qt, self.kt, self.vt, self.row_ptr, self.col_idx, self.work_order,
                       self.ot, self.lse, sched, trace, self.workspace, stream)
+        sba_unreorder(h, self.ot, o, self.workspace, stream)
+        return o
+
+    def lowbit(self, q, k, v, top_p, top_k: int, o=None, trace=None, stream=None):
+        """The same path with the low-bit P.V product: values smoothed and
+        quantised by sba_smooth_v, attention by sba_attention_lowbit."""
+        import torch
+        p = self.plan
+        h = p.handle
+        inf = p.info
+        dev = self.qt.device
+        if not hasattr(self, "vq"):
+            self.vq = torch.empty(p.B, p.H, inf.nb, p.d, inf.bs, dtype=torch.uint8, device=dev)
+            self.vmean = torch.empty(p.B, p.H, inf.nb, p.d, dtype=torch.float32, device=dev)
+            self.vexp = torch.empty(p.B, p.H, dtype=torch.int32, device=dev)
+            nbytes = sba_lowbit_scratch_bytes(h)
+            self.lowbit_scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        if o is None:
+            o = torch.empty_like(q)
+        top_p = list(top_p) if len(top_p) == p.H else [float(top_p[0])] * p.H
+        sba_reorder(h, q, k, v, self.qt, self.kt, self.vt, self.workspace, stream)
+        sba_build_mask(h, self.qt, self.kt, top_p, top_k, self.bitmask, self.row_cnt,
+                       self.row_ptr, self.col_idx, self.work_order, self.workspace, stream)
+        sba_smooth_v(h, self.vt, self.vq, self.vmean, self.vexp, self.workspace, stream)
+        sba_attention_lowbit(h, self.qt, self.kt, self.vq, self.vmean, self.vexp, self.row_ptr,
+                             self.col_idx, self.work_order, self.ot, self.lse, trace,
+                             self.lowbit_scratch, self.lowbit_scratch.numel(), self.workspace,
+                             stream)
         sba_unreorder(h, self.ot, o, self.workspace, stream)
         return o
 

@@ -53,7 +53,7 @@ namespace {
 
 constexpr int kSmemLimit = 232448;  // 227 KB: opt-in shared memory per CTA
 
-template <int D, int BS>
+template <int D, int BS, bool LB = false>
 struct Cfg {
   static constexpr int M = 128;
   // softmax column groups: 2 (measured best for 128x128 tiles: 64 S columns
@@ -68,17 +68,23 @@ struct Cfg {
   static constexpr int NSB = 3;          // S buffers in TMEM
   static constexpr int PANELS = D / 64;  // 128-byte column panels along d
   static constexpr int Q_BYTES = M * D * 2;
-  static constexpr int TILE_BYTES = BS * D * 2;
+  static constexpr int TILE_BYTES = BS * D * 2;  // a bf16 K (or V) tile
+  // low-bit path (LB): a V tile is bs x d E4M3 codes stored [d][bs]
+  static constexpr int VTILE_BYTES = LB ? BS * D : TILE_BYTES;
   static constexpr int CTRL_BYTES = 10240;  // barriers, ring, masks, row-max exchange
   static constexpr int NT_RAW = (kSmemLimit - 1024 - CTRL_BYTES - Q_BYTES) / TILE_BYTES;
   static constexpr int NT = NT_RAW > 8 ? 8 : NT_RAW;  // K + V slots
-  static constexpr int NK = (NT + 1) / 2, NV = NT - NK;
-  static constexpr int SMEM_USED = 1024 + Q_BYTES + NT * TILE_BYTES + CTRL_BYTES;
+  static constexpr int NK = LB ? 3 : (NT + 1) / 2, NV = LB ? 4 : NT - NK;
+  static constexpr int SMEM_USED = 1024 + Q_BYTES + NK * TILE_BYTES + NV * VTILE_BYTES + CTRL_BYTES;
+  // reference-max threshold (log2 units) beyond which O is rescaled: 2^8 for
+  // bf16 P; 0.75 for E4M3 codes, whose reference sits at 2^8 of the 448 top
+  static constexpr float RESCALE = LB ? 0.75f : 8.0f;
+  static_assert(!LB || (D == 128 && BS == 128), "low-bit path: d = bs = 128");
   // Request at least 120 KB so that only one CTA (one 512-column TMEM
   // allocation) is ever resident per SM.
   static constexpr int SMEM = SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(M, BS, 0, 0);
-  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(M, D, 0, 1);
+  static constexpr uint32_t IDESC_PV = LB ? idesc_e4m3_f32(M, D) : idesc_bf16_f32(M, D, 0, 1);
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_O = 384;
   // barrier indices
@@ -106,7 +112,15 @@ struct AttnParams {
   int sched;
   uint64_t budget_ns;
   float scale_log2;
+  // low-bit path only
+  const float* vmean;    // [B*H][nb][d] block means of V
+  const int32_t* vexp;   // [B*H] power-of-two exponent of the value codes
+  float* lsum;           // [grid][2][nb][2][128] per-block partial row sums
 };
+
+// 1.5 * 2^23: adding it to a float in [-2^22, 2^22) rounds the float to an
+// integer (nearest even) held in the low mantissa bits.
+constexpr float kCodeMagic = 12582912.0f;
 
 // Wait that ignores the abort flag (used to drain in-flight async work).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t budget_ns,
@@ -126,18 +140,18 @@ __device__ __forceinline__ int block_type(const KGeom& g, int j) {
          (static_cast<int>(tw) == g.nW - 1);
 }
 
-template <int D, int BS>
-__global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
+template <int D, int BS, bool LB>
+__global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams P) {
-  using C = Cfg<D, BS>;
+  using C = Cfg<D, BS, LB>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sQ = sm;
   unsigned char* sK = sm + C::Q_BYTES;
   unsigned char* sV = sK + C::NK * C::TILE_BYTES;
-  unsigned char* ctl = sV + C::NV * C::TILE_BYTES;
+  unsigned char* ctl = sV + C::NV * C::VTILE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 516);
@@ -312,10 +326,17 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
           if (!ok) break;
         }
         if (lane == 0) {
-          const uint32_t dst = smem_u32((isv ? sV : sK) + s * C::TILE_BYTES);
-          mbar_arrive_expect_tx(bar(bfull), C::TILE_BYTES);
-          for (int p = 0; p < C::PANELS; ++p)
-            tma_load_2d(dst + p * BS * 128, isv ? &tmV : &tmK, p * 64, rows_base + j * BS, bar(bfull));
+          if (LB && isv) {
+            // E4M3 codes of block j, [d][bs] bytes: one 128-byte-wide box
+            const uint32_t dst = smem_u32(sV + s * C::VTILE_BYTES);
+            mbar_arrive_expect_tx(bar(bfull), C::VTILE_BYTES);
+            tma_load_2d(dst, &tmV, 0, (static_cast<int>(bh) * g.nb + j) * D, bar(bfull));
+          } else {
+            const uint32_t dst = smem_u32((isv ? sV : sK) + s * C::TILE_BYTES);
+            mbar_arrive_expect_tx(bar(bfull), C::TILE_BYTES);
+            for (int p = 0; p < C::PANELS; ++p)
+              tma_load_2d(dst + p * BS * 128, isv ? &tmV : &tmK, p * 64, rows_base + j * BS, bar(bfull));
+          }
         }
         if (isv) {
           ++vt;
@@ -419,11 +440,22 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
         tc_fence_after();
         if (lane == 0) {
           const uint32_t aP = tmem + static_cast<uint32_t>(b) * 128u;
-          const uint32_t v_addr = smem_u32(sV + s * C::TILE_BYTES);
+          if constexpr (LB) {
+            // O += P.V in E4M3: A = P codes in TMEM (8 columns per 32 keys),
+            // B = the block's codes, K-major [d][bs], 32 bytes per k-step
+            const uint32_t v_addr = smem_u32(sV + s * C::VTILE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BS / 16; ++kk) {
-            const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, BS * 128, 1024);
-            mma_ts(tmem + C::COL_O, aP + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BS / 32; ++kk) {
+              const uint64_t bd = smem_desc_sw128(v_addr + kk * 32, 16, 1024);
+              mma_ts_f8(tmem + C::COL_O, aP + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+            }
+          } else {
+            const uint32_t v_addr = smem_u32(sV + s * C::TILE_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BS / 16; ++kk) {
+              const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, BS * 128, 1024);
+              mma_ts(tmem + C::COL_O, aP + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           mma_commit(bar(C::B_PD + b));
           mma_commit(bar(C::B_VE + s));
@@ -523,7 +555,7 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(C::B_X + b));
-          uint32_t pk[CPW / 2];
+          uint32_t pk[LB ? CPW / 4 : CPW / 2];
           float2 acc[4];
           float alpha = 1.f;
           // Exponentials of this group's columns against the reference max.
@@ -542,20 +574,43 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
           }
 #pragma unroll 1
           for (int pass = 0; pass < 2; ++pass) {
-            const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-ref, -ref);
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+            if constexpr (LB) {
+              // ExpCast-FP8 (VC-Attention abstract): the E4M3 code of
+              // 2^(x + 8), x = s*log2(e)/sqrt(d) - ref, is rint(8x + 120):
+              // one multiply-add, the magic add's rounding, a clamp at 0,
+              // and the low byte of each float is a code
+              const float c8 = 8.0f * sl2, bb = 120.0f - 8.0f * ref;
+              const float2 c82 = make_float2(c8, c8), b2 = make_float2(bb, bb);
+              const float2 mg2 = make_float2(kCodeMagic, kCodeMagic);
 #pragma unroll
-            for (int e = 0; e < CPW / 2; ++e) {
-              const float2 x = ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
-              // one pair in eight runs on the FMA pipe to offload MUFU
-              const float2 pp = ((e & 7) == 5) ? exp2_poly2(x)
-                                               : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-              pk[e] = pack_bf16x2(pp.x, pp.y);
-              // row sum of the bf16 values the P.V product uses, so that each
-              // output row is an exact convex combination of V rows
-              acc[e & 3] = fadd2(acc[e & 3], make_float2(__uint_as_float(pk[e] << 16),
-                                                         __uint_as_float(pk[e] & 0xFFFF0000u)));
+              for (int e = 0; e < CPW / 4; ++e) {
+                const float2 y0 = fadd2(ffma2(make_float2(s[4 * e], s[4 * e + 1]), c82, b2), mg2);
+                const float2 y1 =
+                    fadd2(ffma2(make_float2(s[4 * e + 2], s[4 * e + 3]), c82, b2), mg2);
+                const uint32_t z0 = __float_as_uint(fmaxf(y0.x, kCodeMagic));
+                const uint32_t z1 = __float_as_uint(fmaxf(y0.y, kCodeMagic));
+                const uint32_t z2 = __float_as_uint(fmaxf(y1.x, kCodeMagic));
+                const uint32_t z3 = __float_as_uint(fmaxf(y1.y, kCodeMagic));
+                pk[e] = __byte_perm(__byte_perm(z0, z1, 0x0040), __byte_perm(z2, z3, 0x0040), 0x5410);
+                // row sum of the decoded codes the P.V product uses
+                add_e4m3x4_f32(pk[e], acc[e & 3].x, acc[e & 3].y);
+              }
+            } else {
+              const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-ref, -ref);
+#pragma unroll
+              for (int e = 0; e < CPW / 2; ++e) {
+                const float2 x = ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+                // one pair in eight runs on the FMA pipe to offload MUFU
+                const float2 pp = ((e & 7) == 5) ? exp2_poly2(x)
+                                                 : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                pk[e] = pack_bf16x2(pp.x, pp.y);
+                // row sum of the bf16 values the P.V product uses, so that each
+                // output row is an exact convex combination of V rows
+                acc[e & 3] = fadd2(acc[e & 3], make_float2(__uint_as_float(pk[e] << 16),
+                                                           __uint_as_float(pk[e] & 0xFFFF0000u)));
+              }
             }
             if (i == 0 || pass == 1) break;
             ok = wwait(C::B_X + b, ph);
@@ -564,7 +619,7 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
 #pragma unroll
             for (int k = 1; k < NWG; ++k) mx = fmaxf(mx, xm[k * 128 + t]);
             const float mblk = mx * sl2;
-            const bool grow = mblk > m + 8.0f;
+            const bool grow = mblk > m + C::RESCALE;
             if (!__any_sync(0xffffffffu, grow)) break;
             const float m_new = grow ? mblk : m;
             alpha = grow ? ex2_approx(m - m_new) : 1.f;
@@ -589,17 +644,31 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           l *= alpha;
-          // P (bf16 pairs) over the first half of this group's S columns
-          const uint32_t pcol = scol + wg * (CPW / 2);
-          if constexpr (CPW >= 64) {
+          const float lblk = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                             ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+          if constexpr (LB) {
+            // E4M3 codes (4 per column) over this group's quarter of S
+            tmem_st16(scol + wg * (CPW / 4), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+            P.lsum[((static_cast<size_t>(blockIdx.x * 2 + (ouses & 1)) * g.nb + i) * 2 + wg) * 128 + t] =
+                lblk;
+          } else if constexpr (CPW >= 64) {
+            // P (bf16 pairs) over the first half of this group's S columns
+            const uint32_t pcol = scol + wg * (CPW / 2);
 #pragma unroll
             for (int c = 0; c < CPW / 64; ++c)
               tmem_st32(pcol + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
           } else {
-            tmem_st16(pcol, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+            tmem_st16(scol + wg * (CPW / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
           }
-          l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-               ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+          l += lblk;
+          if constexpr (LB) {
+            // after a rescale, the row's earlier per-block sums share the old reference
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+              float* lp = P.lsum + (static_cast<size_t>(blockIdx.x * 2 + (ouses & 1)) * g.nb) * 256 +
+                          wg * 128 + t;
+              for (int q = 0; q < i; ++q) lp[q * 256] *= alpha;
+            }
+          }
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(bar(C::B_PR + b));
@@ -627,6 +696,36 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
         float lt = xsum[t];
 #pragma unroll
         for (int k = 1; k < NWG; ++k) lt += xsum[k * 128 + t];
+        if constexpr (LB) {
+          // V-Smooth: O = (2^e * P.codes + sum_j l_j mu_j) / l, with l_j the
+          // row's per-block sums of both groups
+          const float sig = ldexpf(1.0f, __ldg(&P.vexp[bh]));
+          const float* lp = P.lsum + (static_cast<size_t>(blockIdx.x * 2 + ((ouses - 1) & 1)) * g.nb) * 256 + t;
+#pragma unroll
+          for (int half = 0; half < DPW; half += 32) {  // 32 columns at a time
+            float mt[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) mt[c] = 0.f;
+            for (int q = 0; q < n; ++q) {
+              int j = __ldg(&P.col_idx[start + q]);
+              j = (j < 0 || j >= g.nb) ? 0 : j;
+              const float lj = lp[q * 256] + lp[q * 256 + 128];
+              const float4* mu = reinterpret_cast<const float4*>(
+                  P.vmean + (static_cast<size_t>(bh) * g.nb + j) * D + wg * DPW + half);
+#pragma unroll
+              for (int c4 = 0; c4 < 8; ++c4) {
+                const float4 u = __ldg(&mu[c4]);
+                mt[4 * c4 + 0] = fmaf(lj, u.x, mt[4 * c4 + 0]);
+                mt[4 * c4 + 1] = fmaf(lj, u.y, mt[4 * c4 + 1]);
+                mt[4 * c4 + 2] = fmaf(lj, u.z, mt[4 * c4 + 2]);
+                mt[4 * c4 + 3] = fmaf(lj, u.w, mt[4 * c4 + 3]);
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              orr[half + c] = __float_as_uint(fmaf(sig, __uint_as_float(orr[half + c]), mt[c]));
+          }
+        }
         if (t < BS) {
           const float inv = qvalid ? 1.0f / lt : 0.f;
 #pragma unroll
@@ -638,7 +737,9 @@ __global__ void __launch_bounds__(Cfg<D, BS>::THREADS, 1)
             v.w = pack_bf16x2(__uint_as_float(orr[c + 6]) * inv, __uint_as_float(orr[c + 7]) * inv);
             *reinterpret_cast<uint4*>(optr + c) = v;
           }
-          if (P.lse && wg == 0) P.lse[orow] = qvalid ? (m * 0.69314718055994531f + logf(lt)) : 0.f;
+          // the low-bit codes carry a factor 2^8 (the reference maps to code 120)
+          const float mref = LB ? m - 8.0f : m;
+          if (P.lse && wg == 0) P.lse[orow] = qvalid ? (mref * 0.69314718055994531f + logf(lt)) : 0.f;
         }
       }
       if (P.trace && threadIdx.x == 0) {
@@ -804,16 +905,31 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int D, int box_r
   return r == CUDA_SUCCESS;
 }
 
+// 8-bit codes [rows][inner] (inner = 128 bytes), boxes of box_rows rows.
+bool make_map_u8(CUtensorMap* map, const void* base, int64_t rows, int inner, int box_rows) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(inner), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int g_grid_size = 0;
 
-template <int D, int BS>
+template <int D, int BS, bool LB = false>
 cudaError_t launch_tc(const sba_plan* p, const void* qt, const void* kt, const void* vt,
                       const AttnParams& ap, cudaStream_t st) {
-  using C = Cfg<D, BS>;
+  using C = Cfg<D, BS, LB>;
   const int64_t rows = static_cast<int64_t>(p->g.B) * p->g.H * p->info.Npad;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, qt, rows, D, 128) || !make_map(&mk, kt, rows, D, BS) ||
-      !make_map(&mv, vt, rows, D, BS)) {
+  const bool vmap = LB ? make_map_u8(&mv, vt, static_cast<int64_t>(p->g.B) * p->g.H * p->info.nb * D, BS, D)
+                       : make_map(&mv, vt, rows, D, BS);
+  if (!make_map(&mq, qt, rows, D, 128) || !make_map(&mk, kt, rows, D, BS) || !vmap) {
     set_error("cuTensorMapEncodeTiled unavailable or rejected the tensor");
     return cudaErrorInvalidValue;
   }
@@ -827,11 +943,11 @@ cudaError_t launch_tc(const sba_plan* p, const void* qt, const void* kt, const v
     set_error("device offers %d bytes of shared memory per CTA, kernel needs %d", optin, C::SMEM);
     return cudaErrorInvalidConfiguration;
   }
-  e = cudaFuncSetAttribute(attn_tc_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  e = cudaFuncSetAttribute(attn_tc_kernel<D, BS, LB>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = ap.sched == SBA_SCHED_LPT ? std::min(sms, ap.R) : ap.R;
   if (ap.sched == SBA_SCHED_LPT) g_grid_size = grid;
-  attn_tc_kernel<D, BS><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, ap);
+  attn_tc_kernel<D, BS, LB><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, ap);
   return cudaGetLastError();
 }
 
@@ -869,10 +985,44 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
   ap.sched = sched;
   ap.budget_ns = p->wait_budget_ns;
   ap.scale_log2 = scale_log2;
+  ap.vmean = nullptr;
+  ap.vexp = nullptr;
+  ap.lsum = nullptr;
   if (g.d == 128 && g.bs == 128) return launch_tc<128, 128>(p, qt, kt, vt, ap, st);
   if (g.d == 128 && g.bs == 64) return launch_tc<128, 64>(p, qt, kt, vt, ap, st);
   if (g.d == 64 && g.bs == 128) return launch_tc<64, 128>(p, qt, kt, vt, ap, st);
   if (g.d == 64 && g.bs == 64) return launch_tc<64, 64>(p, qt, kt, vt, ap, st);
+  return cudaErrorInvalidValue;
+}
+
+size_t lowbit_scratch_bytes(const sba_plan* p, int sms) {
+  return static_cast<size_t>(std::max(1, std::min(sms, p->info.rows))) * 2 * p->info.nb * 2 * 128 *
+         sizeof(float);
+}
+
+cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const void* kt, const void* vq,
+                                    const float* vmean, const int32_t* vexp, const int32_t* row_ptr,
+                                    const int32_t* col_idx, const int32_t* work_order, void* ot,
+                                    float* lse, uint64_t* trace, float* lsum, void* workspace,
+                                    cudaStream_t st) {
+  KGeom g = make_kgeom(p);
+  AttnParams ap;
+  ap.g = g;
+  ap.row_ptr = row_ptr;
+  ap.col_idx = col_idx;
+  ap.work_order = work_order;
+  ap.ot = static_cast<__nv_bfloat16*>(ot);
+  ap.lse = lse;
+  ap.trace = trace;
+  ap.ctrl = reinterpret_cast<Ctrl*>(static_cast<char*>(workspace) + p->ws_ctrl);
+  ap.R = p->info.rows;
+  ap.sched = SBA_SCHED_LPT;
+  ap.budget_ns = p->wait_budget_ns;
+  ap.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(g.d)));
+  ap.vmean = vmean;
+  ap.vexp = vexp;
+  ap.lsum = lsum;
+  if (g.d == 128 && g.bs == 128) return launch_tc<128, 128, true>(p, qt, kt, vq, ap, st);
   return cudaErrorInvalidValue;
 }
 

@@ -239,6 +239,45 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (both K-major)
+// and an fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                   // D: f32; A, B: E4M3 (0)
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= A[tmem] * B[smem] with 8-bit operands (kind::f8f6f4); A is
+// K-major, one row per TMEM lane, four codes per 32-bit column.
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
+      : "memory");
+}
+
+// a += the even-position, b += the odd-position values of the four E4M3
+// codes packed in w (exact widening through f16, one fp32 add each).
+__device__ __forceinline__ void add_e4m3x4_f32(uint32_t w, float& a, float& b) {
+  asm("{\n\t.reg .b16 lo, hi, x0, x1, x2, x3;\n\t.reg .b32 h0, h1;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h0, lo;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h1, hi;\n\t"
+      "mov.b32 {x0, x1}, h0;\n\t"
+      "mov.b32 {x2, x3}, h1;\n\t"
+      "add.rn.f32.f16 %0, x0, %0;\n\t"
+      "add.rn.f32.f16 %1, x1, %1;\n\t"
+      "add.rn.f32.f16 %0, x2, %0;\n\t"
+      "add.rn.f32.f16 %1, x3, %1;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "r"(w));
+}
+
 // Round two floats to bf16 (nearest even) and pack: lo in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -230,6 +230,59 @@ SBA_API sba_status sba_build_stripe_mask(const sba_plan* plan, const sba_stripe*
                                          int32_t* col_idx, int32_t* work_order, void* workspace,
                                          void* stream);
 
+/* Low-bit P.V path (VC-Attention: Value Smoothing and Softmax Casting for
+ * Low-bit Attention, abstract: V-Smooth and ExpCast-FP8). Two calls beside
+ * the bf16 path: sba_smooth_v quantises the values once per layer, and
+ * sba_attention_lowbit runs the same block-sparse attention with E4M3
+ * probabilities and E4M3 values in the P.V product (S = Q.K^T stays bf16).
+ *
+ * sba_smooth_v: V-Smooth. For every key block j of head (b, h):
+ *   mu_j = mean of vt over the block's real tokens (summed in fp64, rounded
+ *   once to fp32); R = vt - mu_j in fp32 (0 on padding slots); one
+ *   power-of-two scale per head, 2^e with e the smallest integer such that
+ *   max|R| <= 448 * 2^e (e = 0 when R is all zero); codes = E4M3(R * 2^-e),
+ *   round to nearest even, saturating at +-448, the sign kept on a negative
+ *   value that rounds to zero. (The page's online clustering of value tokens
+ *   is not done: cube blocks already hold spatio-temporal neighbours.)
+ * Inputs: vt, bf16 [B][H][Npad][d] from sba_reorder (16-byte aligned).
+ * Outputs (device, caller-owned): vq uint8 [B][H][nb][d][bs] - each block's
+ *   codes transposed, channel-major (16-byte aligned); vmean fp32
+ *   [B][H][nb][d] (16-byte aligned); vexp int32 [B][H]. workspace as for
+ *   sba_build_mask (its pooled-means area holds per-block maxima meanwhile).
+ * bf16 plans with d <= 128 only (else SBA_ERR_UNSUPPORTED). Deterministic. */
+SBA_API sba_status sba_smooth_v(const sba_plan* plan, const void* vt, void* vq, float* vmean,
+                                int32_t* vexp, void* workspace, void* stream);
+
+/* Bytes of scratch sba_attention_lowbit needs on the current device:
+ * min(SMs, R) * 2 * nb * 2 * 128 * 4 (per persistent CTA, two rows' per-block
+ * partial row sums of both softmax column groups). */
+SBA_API sba_status sba_lowbit_scratch_bytes(const sba_plan* plan, size_t* bytes);
+
+/* Block-sparse attention with ExpCast-FP8 probabilities and V-Smooth values.
+ * Per row (query block i) and selected key block j, on real keys:
+ *   x = q.k / sqrt(d) * log2(e) - m, with m the row's reference maximum: the
+ *     first selected block's row maximum, replaced by a later block's when that
+ *     exceeds it by more than 0.75 (accumulators rescaled);
+ *   code = clamp(rint(8x + 120), 0, 126) (one multiply-add: the E4M3 code of
+ *     ~2^(x+8), linear in the mantissa between powers of two), P = its value;
+ *   A += P . (2^e * codes_j) on the tensor core (kind::f8f6f4, fp32
+ *     accumulation), l_j = sum of P over the block, L += l_j;
+ *   o = (A + sum_j l_j mu_j) / L, lse = ln(L) + (m - 8) ln(2).
+ * Rows without blocks give o = 0 and lse = -inf; padding query slots 0.
+ * Inputs as for sba_attention with vq, vmean, vexp from sba_smooth_v; the
+ * longest-first persistent scheduler is always used (work_order required).
+ * scratch: device, at least sba_lowbit_scratch_bytes (16-byte aligned).
+ * bf16 plans with d = 128 and bs = 128 only (else SBA_ERR_UNSUPPORTED).
+ * Results are not bit-identical to the bf16 path: E4M3 values carry ~3
+ * mantissa bits, so the output departs from exact attention by a few
+ * percent (measured and reported by the tests). */
+SBA_API sba_status sba_attention_lowbit(const sba_plan* plan, const void* qt, const void* kt,
+                                        const void* vq, const float* vmean, const int32_t* vexp,
+                                        const int32_t* row_ptr, const int32_t* col_idx,
+                                        const int32_t* work_order, void* ot, float* lse,
+                                        uint64_t* trace, void* scratch, size_t scratch_bytes,
+                                        void* workspace, void* stream);
+
 /* Block-sparse attention forward (FVAttn abstract: attention over the
  * materialised mask). For every real query slot q of block i:
  *   o_q = sum_{j in cols(i)} sum_{real keys k of j} softmax(q.k / sqrt(d)) v_k

@@ -181,3 +181,25 @@ def test_stripe_struct_matches_the_header(sba):
     text = open(os.path.join(ROOT, "include", "sba.h")).read()
     assert "int32_t Tw, To, Ts;" in text and "int32_t Sw, So, Ss;" in text
     assert [f[0] for f in sba.sba_stripe._fields_] == ["Tw", "To", "Ts", "Sw", "So", "Ss"]
+
+
+def test_lowbit_calls_validate_before_any_launch(sba):
+    fake = 1 << 20
+    plan64 = sba.Plan(1, 2, 8, 16, 16, 64, (4, 4, 4), "bf16")
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_attention_lowbit(plan64.handle, fake, fake, fake, fake, fake, fake, fake, fake,
+                                 fake, None, None, fake, 1 << 30, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_UNSUPPORTED
+    plan = sba.Plan(1, 2, 5, 20, 19, 128, (2, 8, 8), "bf16")
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_attention_lowbit(plan.handle, fake, fake, fake, fake, fake, fake, fake, None,
+                                 fake, None, None, fake, 1 << 30, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG  # work_order is required
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_attention_lowbit(plan.handle, fake, fake, fake + 8, fake, fake, fake, fake, fake,
+                                 fake, None, None, fake, 1 << 30, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG  # misaligned codes
+    planf = sba.Plan(1, 2, 4, 8, 8, 64, (4, 4, 4), "f32")
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_smooth_v(planf.handle, fake, fake, fake, fake, fake, stream=0)
+    assert e.value.status == sba.SBA_ERR_UNSUPPORTED

@@ -1,0 +1,157 @@
+"""GPU parity of the low-bit P.V path (VC-Attention: Value Smoothing and
+Softmax Casting for Low-bit Attention, abstract: V-Smooth, ExpCast-FP8)
+through the C ABI.
+
+sba_smooth_v is integer work once its fp32 inputs are fixed: codes, block
+means and exponents are compared bit-exactly with the oracle on the GPU's own
+reordered values. sba_attention_lowbit is compared with the oracle's low-bit
+attention on the GPU's CSR and codes within the bf16 tolerance (max-abs
+2e-2, rel-L2 1e-2, lse 1e-2); its departure from exact attention is the
+quantisation error of the method and is only bounded loosely (rel-L2 < 6 %)."""
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from parity_utils import ATOL, REL_L2, attention_errors, geom_of, sample_blocks, to64
+
+pytestmark = pytest.mark.gpu
+
+SMALL = datagen.custom("lowbit_small", 1, 3, 5, 20, 19, 128, (2, 8, 8), top_p=(0.8, 0.9, 0.95),
+                       top_k=3, rope_split=(44, 42, 42))
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _run(wl, seed=0):
+    import block_sparse_attention_sba_b200 as sba
+    dev = torch.device("cuda:0")
+    q, k, v = datagen.generate(wl, seed=seed, device=dev)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube, order=getattr(wl, "order", "cube"))
+    sa = sba.SparseAttention(plan, device=dev)
+    o = sa.lowbit(q, k, v, wl.top_p_per_head(), wl.top_k)
+    torch.cuda.synchronize()
+    status = sa.check()
+    nnz = int(sa.row_ptr[-1].item())
+    return {"status": status, "sa": sa, "o": o.cpu(), "qt": sa.qt.cpu(), "kt": sa.kt.cpu(),
+            "vt": sa.vt.cpu(), "ot": sa.ot.cpu(), "lse": sa.lse.cpu(),
+            "vq": sa.vq.cpu().numpy(), "vmean": sa.vmean.cpu().numpy(),
+            "vexp": sa.vexp.cpu().numpy().astype(np.int64),
+            "row_cnt": sa.row_cnt.cpu().numpy().astype(np.int64),
+            "row_ptr": sa.row_ptr.cpu().numpy().astype(np.int64),
+            "col_idx": sa.col_idx[:nnz].cpu().numpy().astype(np.int64)}
+
+
+def _check_smooth(wl, gpu):
+    g = geom_of(wl)
+    codes, mu, e = oracle.v_smooth(to64(gpu["vt"]), g)
+    B, H = codes.shape[:2]
+    ref_q = codes.reshape(B, H, g.nb, g.bs, -1).transpose(0, 1, 2, 4, 3)  # [.., d, bs]
+    assert np.array_equal(gpu["vexp"], e)
+    assert np.array_equal(gpu["vmean"], mu)
+    assert np.array_equal(gpu["vq"], ref_q)
+    return codes, mu, e
+
+
+def _check_attention(wl, gpu, codes, mu, e, blocks):
+    g = geom_of(wl)
+    valid = oracle.slot_valid(g)
+    ref_rows, got_rows, ref_l, got_l, ex_rows = [], [], [], [], []
+    by_head = {}
+    for (b, h, i) in blocks:
+        by_head.setdefault((b, h), []).append(i)
+    for (b, h), idx in by_head.items():
+        base = (b * wl.H + h) * g.nb
+        rp = gpu["row_ptr"][base:base + g.nb + 1] - gpu["row_ptr"][base]
+        ci = gpu["col_idx"][gpu["row_ptr"][base]:gpu["row_ptr"][base + g.nb]]
+        qt = to64(gpu["qt"][b:b + 1, h:h + 1])
+        kt = to64(gpu["kt"][b:b + 1, h:h + 1])
+        Ot, lse = oracle.attention_fp8(qt, kt, codes[b:b + 1, h:h + 1], mu[b:b + 1, h:h + 1],
+                                       e[b:b + 1, h:h + 1], g, rp, ci, blocks=[(0, 0, i) for i in idx])
+        Ox, _ = oracle.attention(qt, kt, to64(gpu["vt"][b:b + 1, h:h + 1]), g, rp, ci,
+                                 blocks=[(0, 0, i) for i in idx])
+        for i in idx:
+            sl = slice(i * g.bs, (i + 1) * g.bs)
+            m = valid[sl]
+            ref_rows.append(Ot[0, 0, sl][m])
+            ex_rows.append(Ox[0, 0, sl][m])
+            got_rows.append(to64(gpu["ot"][b, h, sl])[m])
+            ref_l.append(lse[0, 0, sl][m])
+            got_l.append(gpu["lse"][b, h, sl].double().numpy()[m])
+    R, G, X = np.concatenate(ref_rows), np.concatenate(got_rows), np.concatenate(ex_rows)
+    mx, rel = attention_errors(G, R)
+    assert mx <= ATOL and rel <= REL_L2, (mx, rel)
+    assert np.abs(np.concatenate(got_l) - np.concatenate(ref_l)).max() <= 1e-2
+    _, rel_exact = attention_errors(G, X)
+    assert rel_exact < 0.06, rel_exact
+    return mx, rel, rel_exact
+
+
+def test_lowbit_small_every_row():
+    _need_gpu()
+    gpu = _run(SMALL)
+    assert gpu["status"] == 0
+    codes, mu, e = _check_smooth(SMALL, gpu)
+    g = geom_of(SMALL)
+    blocks = [(0, h, i) for h in range(SMALL.H) for i in range(g.nb)]
+    _check_attention(SMALL, gpu, codes, mu, e, blocks)
+
+
+def test_lowbit_wan_layer_sampled_rows():
+    """The Wan-shaped layer (40 heads x 308 blocks): smoothing bit-exact on
+    every head, attention on sampled rows of every fourth head."""
+    _need_gpu()
+    wl = datagen.WORKLOADS["wan"]
+    gpu = _run(wl)
+    assert gpu["status"] == 0
+    codes, mu, e = _check_smooth(wl, gpu)
+    blocks = [x for x in sample_blocks(wl, gpu["row_cnt"], per_head=1, seed=5) if x[1] % 4 == 0]
+    _check_attention(wl, gpu, codes, mu, e, blocks)
+
+
+def test_lowbit_empty_rows_and_rejected_shapes():
+    _need_gpu()
+    import block_sparse_attention_sba_b200 as sba
+    wl = SMALL
+    g = geom_of(wl)
+    dev = torch.device("cuda:0")
+    q, k, v = datagen.generate(wl, seed=1, device=dev)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    sa = sba.SparseAttention(plan, device=dev)
+    h = plan.handle
+    sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace)
+    # a stripe mask whose third head keeps nothing: those rows must come out empty
+    sba.sba_build_stripe_mask(h, [(3, -1, 0, 5, -2, 0), (1, 0, 0, 1, 0, 0), (1, 9, 0, 1, 0, 0)],
+                              sa.bitmask, sa.row_cnt, sa.row_ptr, sa.col_idx, sa.work_order,
+                              sa.workspace)
+    vq = torch.empty(1, wl.H, g.nb, wl.d, g.bs, dtype=torch.uint8, device=dev)
+    vmean = torch.empty(1, wl.H, g.nb, wl.d, dtype=torch.float32, device=dev)
+    vexp = torch.empty(1, wl.H, dtype=torch.int32, device=dev)
+    sba.sba_smooth_v(h, sa.vt, vq, vmean, vexp, sa.workspace)
+    nbytes = sba.sba_lowbit_scratch_bytes(h)
+    scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    with pytest.raises(sba.SbaError) as err:
+        sba.sba_attention_lowbit(h, sa.qt, sa.kt, vq, vmean, vexp, sa.row_ptr, sa.col_idx,
+                                 sa.work_order, sa.ot, sa.lse, None, scratch, nbytes - 16,
+                                 sa.workspace)
+    assert err.value.status == sba.SBA_ERR_CAPACITY
+    sba.sba_attention_lowbit(h, sa.qt, sa.kt, vq, vmean, vexp, sa.row_ptr, sa.col_idx,
+                             sa.work_order, sa.ot, sa.lse, None, scratch, nbytes, sa.workspace)
+    torch.cuda.synchronize()
+    assert sa.check() == 0
+    valid = oracle.slot_valid(g)
+    ot = sa.ot.cpu()
+    lse = sa.lse.cpu().double().numpy()
+    assert torch.all(ot[0, 2] == 0)
+    assert np.all(np.isneginf(lse[0, 2][valid]))
+    assert torch.isfinite(ot[0, :2].float()).all()
+    plan64 = sba.Plan(1, 2, 8, 16, 16, 64, (4, 4, 4), "bf16")
+    with pytest.raises(sba.SbaError) as err:
+        sba.sba_attention_lowbit(plan64.handle, sa.qt, sa.kt, vq, vmean, vexp, sa.row_ptr,
+                                 sa.col_idx, sa.work_order, sa.ot, sa.lse, None, scratch, nbytes,
+                                 sa.workspace)
+    assert err.value.status == sba.SBA_ERR_UNSUPPORTED
