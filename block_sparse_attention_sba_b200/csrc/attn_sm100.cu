@@ -32,8 +32,13 @@
 //   warp  4*NWG+2        P.V issuer (one thread)
 // TMEM: S buffers at columns 0, 128, 256; O at 384.
 // Rescaling of O is skipped while the running row max grows by less than
-// 2^8 (the final normalisation uses the same reference max, so the result is
-// exact up to rounding); padding keys of edge cubes are masked to -inf.
+// 2^24 (the final normalisation uses the same reference max, so the result is
+// exact up to rounding; bf16 P up to 2^24 stays far inside fp32 range for O
+// and the row sum); padding keys of edge cubes are masked to -inf.
+// Low-bit variant (LB, VC-Attention abstract): E4M3 probability codes from
+// one multiply-add (ExpCast-FP8), O += P.V as an 8-bit tensor-core product
+// on V-Smooth codes, per-block row sums kept with their reference for the
+// block-mean term; the reference moves when a block exceeds it by 2^2.75.
 // Scheduler: SBA_SCHED_LPT launches one persistent CTA per SM that takes rows
 // in longest-first work order from an atomic counter (the counter resets
 // itself when the last CTA exits); SBA_SCHED_HEAD_MAJOR launches one CTA per
@@ -76,9 +81,12 @@ struct Cfg {
   static constexpr int NT = NT_RAW > 8 ? 8 : NT_RAW;  // K + V slots
   static constexpr int NK = LB ? 3 : (NT + 1) / 2, NV = LB ? 4 : NT - NK;
   static constexpr int SMEM_USED = 1024 + Q_BYTES + NK * TILE_BYTES + NV * VTILE_BYTES + CTRL_BYTES;
-  // reference-max threshold (log2 units) beyond which O is rescaled: 2^8 for
-  // bf16 P; 0.75 for E4M3 codes, whose reference sits at 2^8 of the 448 top
-  static constexpr float RESCALE = LB ? 0.75f : 8.0f;
+  // reference-max threshold (log2 units) beyond which O is rescaled. bf16
+  // P up to 2^24 keeps O and the row sum far inside fp32 range and makes a
+  // rescale rare (the running maximum of a row rarely jumps that far); E4M3
+  // codes have 2.75 octaves of headroom above the reference (code 104 of 126).
+  static constexpr float RESCALE = LB ? 2.75f : 24.0f;
+  static constexpr float LB_BIAS = 104.0f;  // E4M3 code of the reference
   static_assert(!LB || (D == 128 && BS == 128), "low-bit path: d = bs = 128");
   // Request at least 120 KB so that only one CTA (one 512-column TMEM
   // allocation) is ever resident per SM.
@@ -115,7 +123,7 @@ struct AttnParams {
   // low-bit path only
   const float* vmean;    // [B*H][nb][d] block means of V
   const int32_t* vexp;   // [B*H] power-of-two exponent of the value codes
-  float* lsum;           // [grid][2][nb][2][128] per-block partial row sums
+  float* lsum;           // float2 [grid][2][nb][2][128]: per-block partial row sum, its reference
 };
 
 // 1.5 * 2^23: adding it to a float in [-2^22, 2^22) rounds the float to an
@@ -560,7 +568,7 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           float alpha = 1.f;
           // Exponentials of this group's columns against the reference max.
           // After the first block the running max is used speculatively
-          // (the usual case: no group's maximum exceeds it by more than 2^8)
+          // (the usual case: no group's maximum exceeds it by more than RESCALE)
           // while the exchange completes; the rare block that does exceed it
           // rescales O and goes round once more with the new reference.
           float ref = m;
@@ -578,10 +586,10 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
             for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
             if constexpr (LB) {
               // ExpCast-FP8 (VC-Attention abstract): the E4M3 code of
-              // 2^(x + 8), x = s*log2(e)/sqrt(d) - ref, is rint(8x + 120):
+              // 2^(x + 6), x = s*log2(e)/sqrt(d) - ref, is rint(8x + 104):
               // one multiply-add, the magic add's rounding, a clamp at 0,
               // and the low byte of each float is a code
-              const float c8 = 8.0f * sl2, bb = 120.0f - 8.0f * ref;
+              const float c8 = 8.0f * sl2, bb = C::LB_BIAS - 8.0f * ref;
               const float2 c82 = make_float2(c8, c8), b2 = make_float2(bb, bb);
               const float2 mg2 = make_float2(kCodeMagic, kCodeMagic);
 #pragma unroll
@@ -649,8 +657,9 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           if constexpr (LB) {
             // E4M3 codes (4 per column) over this group's quarter of S
             tmem_st16(scol + wg * (CPW / 4), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-            P.lsum[((static_cast<size_t>(blockIdx.x * 2 + (ouses & 1)) * g.nb + i) * 2 + wg) * 128 + t] =
-                lblk;
+            // this block's partial row sum and the reference it is relative to
+            reinterpret_cast<float2*>(P.lsum)[((static_cast<size_t>(blockIdx.x * 2 + (ouses & 1)) * g.nb + i) * 2 + wg) * 128 + t] =
+                make_float2(lblk, m);
           } else if constexpr (CPW >= 64) {
             // P (bf16 pairs) over the first half of this group's S columns
             const uint32_t pcol = scol + wg * (CPW / 2);
@@ -661,14 +670,6 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
             tmem_st16(scol + wg * (CPW / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
           }
           l += lblk;
-          if constexpr (LB) {
-            // after a rescale, the row's earlier per-block sums share the old reference
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
-              float* lp = P.lsum + (static_cast<size_t>(blockIdx.x * 2 + (ouses & 1)) * g.nb) * 256 +
-                          wg * 128 + t;
-              for (int q = 0; q < i; ++q) lp[q * 256] *= alpha;
-            }
-          }
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(bar(C::B_PR + b));
@@ -700,7 +701,8 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           // V-Smooth: O = (2^e * P.codes + sum_j l_j mu_j) / l, with l_j the
           // row's per-block sums of both groups
           const float sig = ldexpf(1.0f, __ldg(&P.vexp[bh]));
-          const float* lp = P.lsum + (static_cast<size_t>(blockIdx.x * 2 + ((ouses - 1) & 1)) * g.nb) * 256 + t;
+          const float2* lp = reinterpret_cast<const float2*>(P.lsum) +
+                             (static_cast<size_t>(blockIdx.x * 2 + ((ouses - 1) & 1)) * g.nb) * 256 + t;
 #pragma unroll
           for (int half = 0; half < DPW; half += 32) {  // 32 columns at a time
             float mt[32];
@@ -709,7 +711,9 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
             for (int q = 0; q < n; ++q) {
               int j = __ldg(&P.col_idx[start + q]);
               j = (j < 0 || j >= g.nb) ? 0 : j;
-              const float lj = lp[q * 256] + lp[q * 256 + 128];
+              // both groups' partial sums, brought to the final reference
+              const float2 p0 = lp[q * 256], p1 = lp[q * 256 + 128];
+              const float lj = (p0.x + p1.x) * ex2_approx(p0.y - m);
               const float4* mu = reinterpret_cast<const float4*>(
                   P.vmean + (static_cast<size_t>(bh) * g.nb + j) * D + wg * DPW + half);
 #pragma unroll
@@ -737,8 +741,8 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
             v.w = pack_bf16x2(__uint_as_float(orr[c + 6]) * inv, __uint_as_float(orr[c + 7]) * inv);
             *reinterpret_cast<uint4*>(optr + c) = v;
           }
-          // the low-bit codes carry a factor 2^8 (the reference maps to code 120)
-          const float mref = LB ? m - 8.0f : m;
+          // the low-bit codes carry a factor 2^6 (the reference maps to code 104)
+          const float mref = LB ? m - 6.0f : m;
           if (P.lse && wg == 0) P.lse[orow] = qvalid ? (mref * 0.69314718055994531f + logf(lt)) : 0.f;
         }
       }
@@ -997,7 +1001,7 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
 
 size_t lowbit_scratch_bytes(const sba_plan* p, int sms) {
   return static_cast<size_t>(std::max(1, std::min(sms, p->info.rows))) * 2 * p->info.nb * 2 * 128 *
-         sizeof(float);
+         sizeof(float2);
 }
 
 cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const void* kt, const void* vq,

@@ -254,20 +254,20 @@ SBA_API sba_status sba_smooth_v(const sba_plan* plan, const void* vt, void* vq, 
                                 int32_t* vexp, void* workspace, void* stream);
 
 /* Bytes of scratch sba_attention_lowbit needs on the current device:
- * min(SMs, R) * 2 * nb * 2 * 128 * 4 (per persistent CTA, two rows' per-block
- * partial row sums of both softmax column groups). */
+ * min(SMs, R) * 2 * nb * 2 * 128 * 8 (per persistent CTA and two rows: per
+ * block and softmax column group, a partial row sum and its reference). */
 SBA_API sba_status sba_lowbit_scratch_bytes(const sba_plan* plan, size_t* bytes);
 
 /* Block-sparse attention with ExpCast-FP8 probabilities and V-Smooth values.
  * Per row (query block i) and selected key block j, on real keys:
  *   x = q.k / sqrt(d) * log2(e) - m, with m the row's reference maximum: the
  *     first selected block's row maximum, replaced by a later block's when that
- *     exceeds it by more than 0.75 (accumulators rescaled);
- *   code = clamp(rint(8x + 120), 0, 126) (one multiply-add: the E4M3 code of
- *     ~2^(x+8), linear in the mantissa between powers of two), P = its value;
+ *     exceeds it by more than 2.75 (accumulators rescaled);
+ *   code = clamp(rint(8x + 104), 0, 126) (one multiply-add: the E4M3 code of
+ *     ~2^(x+6), linear in the mantissa between powers of two), P = its value;
  *   A += P . (2^e * codes_j) on the tensor core (kind::f8f6f4, fp32
  *     accumulation), l_j = sum of P over the block, L += l_j;
- *   o = (A + sum_j l_j mu_j) / L, lse = ln(L) + (m - 8) ln(2).
+ *   o = (A + sum_j l_j mu_j) / L, lse = ln(L) + (m - 6) ln(2).
  * Rows without blocks give o = 0 and lse = -inf; padding query slots 0.
  * Inputs as for sba_attention with vq, vmean, vexp from sba_smooth_v; the
  * longest-first persistent scheduler is always used (work_order required).

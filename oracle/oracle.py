@@ -488,14 +488,15 @@ def stripe_mask(g: Geom, params, B: int) -> dict:
 #   hold spatio-temporal neighbours.
 # * ExpCast-FP8: the probability code of a log2-domain score x taken relative
 #   to the row's reference maximum (x <= 0 at the reference) is
-#   c = clamp(rint(8x + 120), 0, 126): one multiply-add puts the integer part
-#   of x + 15 into the exponent field and eighths of its fraction into the
-#   mantissa field, so decode(c) interpolates 2^(x+8) linearly between powers
-#   of two (exact where 8x is an integer and -14 <= x <= 0). The reference
-#   maps to 2^8 rather than 1 so that normal codes cover 14 octaves below the
-#   maximum; the factor cancels in the normalisation and lse removes it.
+#   c = clamp(rint(8x + 104), 0, 126): one multiply-add puts the integer part
+#   of x + 13 into the exponent field and eighths of its fraction into the
+#   mantissa field, so decode(c) interpolates 2^(x+6) linearly between powers
+#   of two (exact where 8x is an integer and -12 <= x <= 2.75). The reference
+#   maps to 2^6 rather than 1 so that normal codes cover 12 octaves below it
+#   and 2.75 above it; the factor cancels in the normalisation and lse
+#   removes it.
 # * Reference maximum: the row maximum of the first selected block; a later
-#   block whose maximum exceeds the reference by more than 0.75 (log2 units)
+#   block whose maximum exceeds the reference by more than 2.75 (log2 units)
 #   replaces it (the accumulators are rescaled by 2^(old - new)), so that no
 #   code exceeds 126. With low-bit codes the reference changes the result, so
 #   this rule is part of the definition.
@@ -531,8 +532,8 @@ def e4m3_encode(x) -> np.ndarray:
     return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
 
 
-EXPCAST_BIAS = 120.0  # code of the reference maximum (value 2^8)
-EXPCAST_TAU = 0.75    # reference replacement threshold, log2 units
+EXPCAST_BIAS = 104.0  # code of the reference maximum (value 2^6)
+EXPCAST_TAU = 2.75    # reference replacement threshold, log2 units (8 * 2.75 + 104 = 126)
 
 
 def expcast_code(x) -> np.ndarray:
@@ -589,7 +590,7 @@ def attention_fp8(Qt, Kt, codes, mu, e, g: Geom, row_ptr, col_idx, blocks=None):
     - m, probabilities P = decode(expcast_code(x)), l_j = sum of P over the
     block; accumulators A += P @ (sigma * decode(codes_j)), L += l_j,
     M += l_j * mu_j, all rescaled together when the reference m changes.
-    O = (A + M) / L, lse = ln(L) + (m - 8) * ln(2). Padding query slots:
+    O = (A + M) / L, lse = ln(L) + (m - 6) * ln(2). Padding query slots:
     O = 0, lse = 0. Returns (Ot, lse) like ``attention``."""
     Qt = np.asarray(Qt, dtype=np.float64)
     Kt = np.asarray(Kt, dtype=np.float64)
@@ -634,7 +635,7 @@ def attention_fp8(Qt, Kt, codes, mu, e, g: Geom, row_ptr, col_idx, blocks=None):
         qv = valid[q_slots]
         with np.errstate(divide="ignore", invalid="ignore"):
             o = (A + M) / L[:, None]
-            ls = np.log(L) + (m - 8.0) * math.log(2.0)
+            ls = np.log(L) + (m - (EXPCAST_BIAS - 56.0) / 8.0) * math.log(2.0)
         o[~qv] = 0.0
         ls[~qv] = 0.0
         Ot[b, h, q_slots] = o

@@ -614,14 +614,15 @@ def test_e4m3_encode_matches_torch_in_range_and_saturates():
 
 
 def test_expcast_code_closed_forms():
-    k = np.arange(-14, 1)
-    assert np.array_equal(_o.e4m3_decode(_o.expcast_code(k)), np.exp2(k + 8.0))
-    assert _o.expcast_code([0.0, 0.75, -np.inf, np.nan, -50.0, 1.0, 100.0]).tolist() == \
-        [120, 126, 0, 0, 0, 126, 126]
-    x = np.linspace(-14, 0.75, 20001)
+    k = np.arange(-12, 3)
+    assert np.array_equal(_o.e4m3_decode(_o.expcast_code(k)), np.exp2(k + 6.0))
+    assert _o.expcast_code([0.0, 2.75, -np.inf, np.nan, -50.0, 3.0, 100.0]).tolist() == \
+        [104, 126, 0, 0, 0, 126, 126]
+    assert 8 * _o.EXPCAST_TAU + _o.EXPCAST_BIAS == 126  # no code clips below the threshold
+    x = np.linspace(-12, 2.75, 20001)
     c = _o.expcast_code(x)
     assert np.all(np.diff(c) >= 0)                      # monotone
-    rel = _o.e4m3_decode(c) / np.exp2(x + 8.0) - 1.0
+    rel = _o.e4m3_decode(c) / np.exp2(x + 6.0) - 1.0
     # piecewise-linear 2^x (at most +8.61 % at fraction 1/ln2 - 1) and rounding
     # to eighths (a factor 2^(+-1/16)) bound the relative error
     assert rel.max() <= (1 + 0.0861) * 2 ** (1 / 16) - 1 + 1e-9
