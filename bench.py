@@ -47,6 +47,7 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sched-report", action="store_true")
+    ap.add_argument("--no-lowbit", action="store_true", help="skip the low-bit P.V measurement")
     ap.add_argument("--report-all", action="store_true",
                     help="per-call timings, rooflines, density and SM idle for every workload "
                          "(one JSON line each; not the benchmark line)")
@@ -444,6 +445,37 @@ def run_ours(args):
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": ho.numel() * ho.element_size()}
 
+    # the low-bit P.V path (E4M3 probabilities and values) on the same inputs:
+    # informational, not the headline (reduced precision)
+    lowbit = None
+    if not args.no_lowbit and wl.dtype == "bf16" and wl.d == 128 and plan.info.bs == 128:
+        ref_ot = sa.ot.float().clone()
+        sa.lowbit(q, k, v, top_p, wl.top_k, o=o, stream=stream)
+        torch.cuda.synchronize(dev)
+        got = sa.ot.float()
+        rel = float((got - ref_ot).norm() / ref_ot.norm())
+        h = plan.handle
+        t_s, t_a = [], []
+        for _ in range(6):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            flush.zero_()
+            ev[0].record(stream)
+            sba.sba_smooth_v(h, sa.vt, sa.vq, sa.vmean, sa.vexp, sa.workspace, stream)
+            ev[1].record(stream)
+            sba.sba_attention_lowbit(h, sa.qt, sa.kt, sa.vq, sa.vmean, sa.vexp, sa.row_ptr,
+                                     sa.col_idx, sa.work_order, sa.ot, sa.lse, None,
+                                     sa.lowbit_scratch, sa.lowbit_scratch.numel(), sa.workspace,
+                                     stream)
+            ev[2].record(stream)
+            torch.cuda.synchronize(dev)
+            t_s.append(ev[0].elapsed_time(ev[1]))
+            t_a.append(ev[1].elapsed_time(ev[2]))
+        ms_a = statistics.mean(t_a[2:])
+        lowbit = {"ms_smooth_v": round(statistics.mean(t_s[2:]), 4), "ms_attention": round(ms_a, 4),
+                  "tflops_tile": f_tile / (ms_a * 1e-3) / 1e12,
+                  "rel_l2_vs_bf16_output": rel,
+                  "kernel": "attn_tc_kernel<128,128,1> (E4M3 P.V)"}
+
     sched = None
     if not args.no_sched_report:
         sched = sched_report(dev)
@@ -472,7 +504,7 @@ def run_ours(args):
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": f_tile},
-            "scheduler": sched,
+            "scheduler": sched, "lowbit": lowbit,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 7 * args.steps,
             "clocks": clocks, "device_status": sba.sba_status_string(status),
         }
