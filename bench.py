@@ -463,8 +463,7 @@ def run_ours(args):
             sba.sba_smooth_v(h, sa.vt, sa.vq, sa.vmean, sa.vexp, sa.workspace, stream)
             ev[1].record(stream)
             sba.sba_attention_lowbit(h, sa.qt, sa.kt, sa.vq, sa.vmean, sa.vexp, sa.row_ptr,
-                                     sa.col_idx, sa.work_order, sa.ot, sa.lse, None,
-                                     sa.lowbit_scratch, sa.lowbit_scratch.numel(), sa.workspace,
+                                     sa.col_idx, sa.work_order, sa.ot, sa.lse, None, sa.workspace,
                                      stream)
             ev[2].record(stream)
             torch.cuda.synchronize(dev)

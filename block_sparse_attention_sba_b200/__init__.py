@@ -42,7 +42,7 @@ EXPORTED = ["sba_plan_create", "sba_plan_destroy", "sba_plan_query", "sba_worksp
             "sba_check_device_status", "sba_debug_timeout_probe", "sba_perm_export",
             "sba_attention_grid_size", "sba_status_string", "sba_last_error",
             "sba_build_mask_noalloc", "sba_build_stripe_mask", "sba_smooth_v",
-            "sba_lowbit_scratch_bytes", "sba_attention_lowbit"]
+            "sba_attention_lowbit"]
 
 
 class sba_geometry(ctypes.Structure):
@@ -82,9 +82,7 @@ _sig = {
                                _vp, _vp, _vp],
     "sba_build_stripe_mask": [_vp, ctypes.POINTER(sba_stripe), _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "sba_smooth_v": [_vp, _vp, _vp, _vp, _vp, _vp, _vp],
-    "sba_lowbit_scratch_bytes": [_vp, ctypes.POINTER(ctypes.c_size_t)],
-    "sba_attention_lowbit": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
-                             ctypes.c_size_t, _vp, _vp],
+    "sba_attention_lowbit": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "sba_check_device_status": [_vp, _vp, _vp],
     "sba_debug_timeout_probe": [_vp, _vp, ctypes.c_uint64, _vp],
     "sba_perm_export": [_vp, ctypes.POINTER(ctypes.c_int32)],
@@ -197,19 +195,12 @@ def sba_smooth_v(plan: int, vt, vq, vmean, vexp, workspace, stream=None) -> None
                              _stream(stream)), "sba_smooth_v")
 
 
-def sba_lowbit_scratch_bytes(plan: int) -> int:
-    out = ctypes.c_size_t(0)
-    _check(_lib.sba_lowbit_scratch_bytes(plan, ctypes.byref(out)), "sba_lowbit_scratch_bytes")
-    return int(out.value)
-
-
 def sba_attention_lowbit(plan: int, qt, kt, vq, vmean, vexp, row_ptr, col_idx, work_order, ot,
-                         lse=None, trace=None, scratch=None, scratch_bytes: int = 0,
-                         workspace=None, stream=None) -> None:
+                         lse=None, trace=None, workspace=None, stream=None) -> None:
     _check(_lib.sba_attention_lowbit(plan, _ptr(qt), _ptr(kt), _ptr(vq), _ptr(vmean), _ptr(vexp),
                                      _ptr(row_ptr), _ptr(col_idx), _ptr(work_order), _ptr(ot),
-                                     _ptr(lse), _ptr(trace), _ptr(scratch), int(scratch_bytes),
-                                     _ptr(workspace), _stream(stream)), "sba_attention_lowbit")
+                                     _ptr(lse), _ptr(trace), _ptr(workspace), _stream(stream)),
+           "sba_attention_lowbit")
 
 
 def sba_attention(plan: int, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse=None,
@@ -353,8 +344,6 @@ class SparseAttention:
             self.vq = torch.empty(p.B, p.H, inf.nb, p.d, inf.bs, dtype=torch.uint8, device=dev)
             self.vmean = torch.empty(p.B, p.H, inf.nb, p.d, dtype=torch.float32, device=dev)
             self.vexp = torch.empty(p.B, p.H, dtype=torch.int32, device=dev)
-            nbytes = sba_lowbit_scratch_bytes(h)
-            self.lowbit_scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         if o is None:
             o = torch.empty_like(q)
         top_p = list(top_p) if len(top_p) == p.H else [float(top_p[0])] * p.H
@@ -364,8 +353,7 @@ class SparseAttention:
         sba_smooth_v(h, self.vt, self.vq, self.vmean, self.vexp, self.workspace, stream)
         sba_attention_lowbit(h, self.qt, self.kt, self.vq, self.vmean, self.vexp, self.row_ptr,
                              self.col_idx, self.work_order, self.ot, self.lse, trace,
-                             self.lowbit_scratch, self.lowbit_scratch.numel(), self.workspace,
-                             stream)
+                             self.workspace, stream)
         sba_unreorder(h, self.ot, o, self.workspace, stream)
         return o
 

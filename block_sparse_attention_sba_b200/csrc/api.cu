@@ -324,45 +324,21 @@ sba_status sba_smooth_v(const sba_plan* plan, const void* vt, void* vq, float* v
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_smooth_v launch");
 }
 
-static int device_sms() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return sms;
-}
-
-sba_status sba_lowbit_scratch_bytes(const sba_plan* plan, size_t* bytes) {
-  g_err[0] = '\0';
-  if (!plan || !bytes) return fail(SBA_ERR_INVALID_ARG, "plan and bytes must be non-NULL");
-  const int sms = device_sms();
-  if (sms <= 0) return fail(SBA_ERR_CUDA, "cannot read the device's multiprocessor count");
-  *bytes = lowbit_scratch_bytes(plan, sms);
-  return SBA_OK;
-}
-
 sba_status sba_attention_lowbit(const sba_plan* plan, const void* qt, const void* kt, const void* vq,
                                 const float* vmean, const int32_t* vexp, const int32_t* row_ptr,
                                 const int32_t* col_idx, const int32_t* work_order, void* ot,
-                                float* lse, uint64_t* trace, void* scratch, size_t scratch_bytes,
-                                void* workspace, void* stream) {
+                                float* lse, uint64_t* trace, void* workspace, void* stream) {
   g_err[0] = '\0';
   if (!plan || !qt || !kt || !vq || !vmean || !vexp || !row_ptr || !col_idx || !work_order || !ot ||
-      !scratch || !workspace)
+      !workspace)
     return fail(SBA_ERR_INVALID_ARG, "sba_attention_lowbit: NULL argument");
   if (plan->g.dtype != SBA_BF16 || plan->g.d != 128 || plan->info.bs != 128)
     return fail(SBA_ERR_UNSUPPORTED, "sba_attention_lowbit: bf16 plans with d = bs = 128 only");
   if (!aligned16(qt) || !aligned16(kt) || !aligned16(vq) || !aligned16(vmean) || !aligned16(ot) ||
-      !aligned16(scratch) || !aligned16(workspace))
-    return fail(SBA_ERR_INVALID_ARG, "qt, kt, vq, vmean, ot, scratch and workspace must be 16-byte aligned");
-  const int sms = device_sms();
-  if (sms <= 0) return fail(SBA_ERR_CUDA, "cannot read the device's multiprocessor count");
-  const size_t need = lowbit_scratch_bytes(plan, sms);
-  if (scratch_bytes < need)
-    return fail(SBA_ERR_CAPACITY, "scratch of %zu bytes; sba_attention_lowbit needs %zu", scratch_bytes,
-                need);
+      !aligned16(workspace))
+    return fail(SBA_ERR_INVALID_ARG, "qt, kt, vq, vmean, ot and workspace must be 16-byte aligned");
   cudaError_t e = launch_attention_lowbit(plan, qt, kt, vq, vmean, vexp, row_ptr, col_idx, work_order,
-                                          ot, lse, trace, static_cast<float*>(scratch), workspace,
-                                          static_cast<cudaStream_t>(stream));
+                                          ot, lse, trace, workspace, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_attention_lowbit launch");
 }
 

@@ -37,8 +37,9 @@
 // and the row sum); padding keys of edge cubes are masked to -inf.
 // Low-bit variant (LB, VC-Attention abstract): E4M3 probability codes from
 // one multiply-add (ExpCast-FP8), O += P.V as an 8-bit tensor-core product
-// on V-Smooth codes, per-block row sums kept with their reference for the
-// block-mean term; the reference moves when a block exceeds it by 2^2.75.
+// on V-Smooth codes, and the block-mean term sum_j l_j mu_j added to O by a
+// small tf32 product per block (A = the two groups' partial row sums, B = the
+// block mean); the reference moves when a block exceeds it by 2^2.75.
 // Scheduler: SBA_SCHED_LPT launches one persistent CTA per SM that takes rows
 // in longest-first work order from an atomic counter (the counter resets
 // itself when the last CTA exits); SBA_SCHED_HEAD_MAJOR launches one CTA per
@@ -70,17 +71,21 @@ struct Cfg {
   static constexpr int THREADS = SM_THREADS + 96;
   static constexpr int WARP_PROD = NWG * 4, WARP_SISS = NWG * 4 + 1, WARP_PVISS = NWG * 4 + 2;
   static_assert(CPW % 32 == 0 && DPW % 32 == 0, "column groups must be multiples of 32");
-  static constexpr int NSB = 3;          // S buffers in TMEM
+  static constexpr int NSB = 3;  // S buffers in TMEM
   static constexpr int PANELS = D / 64;  // 128-byte column panels along d
   static constexpr int Q_BYTES = M * D * 2;
   static constexpr int TILE_BYTES = BS * D * 2;  // a bf16 K (or V) tile
   // low-bit path (LB): a V tile is bs x d E4M3 codes stored [d][bs]
   static constexpr int VTILE_BYTES = LB ? BS * D : TILE_BYTES;
+  // low-bit path: per V slot, the block-mean operand of the tf32 product
+  // O += [l0 l1] [mu/2^e; mu/2^e]: 128 channels x 8 k, K-major, no swizzle
+  static constexpr int MT_BYTES = LB ? 4096 : 0;
   static constexpr int CTRL_BYTES = 10240;  // barriers, ring, masks, row-max exchange
   static constexpr int NT_RAW = (kSmemLimit - 1024 - CTRL_BYTES - Q_BYTES) / TILE_BYTES;
   static constexpr int NT = NT_RAW > 8 ? 8 : NT_RAW;  // K + V slots
   static constexpr int NK = LB ? 3 : (NT + 1) / 2, NV = LB ? 4 : NT - NK;
-  static constexpr int SMEM_USED = 1024 + Q_BYTES + NK * TILE_BYTES + NV * VTILE_BYTES + CTRL_BYTES;
+  static constexpr int SMEM_USED =
+      1024 + Q_BYTES + NK * TILE_BYTES + NV * (VTILE_BYTES + MT_BYTES) + CTRL_BYTES;
   // reference-max threshold (log2 units) beyond which O is rescaled. bf16
   // P up to 2^24 keeps O and the row sum far inside fp32 range and makes a
   // rescale rare (the running maximum of a row rarely jumps that far); E4M3
@@ -95,6 +100,7 @@ struct Cfg {
   static constexpr uint32_t IDESC_PV = LB ? idesc_e4m3_f32(M, D) : idesc_bf16_f32(M, D, 0, 1);
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_O = 384;
+  static constexpr uint32_t IDESC_MEAN = idesc_tf32_f32(M, D);
   // barrier indices
   static constexpr int B_QF = 0, B_QE = 1, B_KF = 2, B_KE = B_KF + NK, B_VF = B_KE + NK,
                        B_VE = B_VF + NV, B_SR = B_VE + NV, B_PR = B_SR + NSB, B_PD = B_PR + NSB,
@@ -123,7 +129,6 @@ struct AttnParams {
   // low-bit path only
   const float* vmean;    // [B*H][nb][d] block means of V
   const int32_t* vexp;   // [B*H] power-of-two exponent of the value codes
-  float* lsum;           // float2 [grid][2][nb][2][128]: per-block partial row sum, its reference
 };
 
 // 1.5 * 2^23: adding it to a float in [-2^22, 2^22) rounds the float to an
@@ -159,7 +164,8 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
   unsigned char* sQ = sm;
   unsigned char* sK = sm + C::Q_BYTES;
   unsigned char* sV = sK + C::NK * C::TILE_BYTES;
-  unsigned char* ctl = sV + C::NV * C::VTILE_BYTES;
+  unsigned char* sMT = sV + C::NV * C::VTILE_BYTES;  // LB: block-mean operands
+  unsigned char* ctl = sMT + C::NV * C::MT_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 516);
@@ -333,6 +339,31 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           ok = wait1(bempty, (r - 1) & 1);
           if (!ok) break;
         }
+        if constexpr (LB) {
+          if (isv) {
+            // block j's mean / 2^e as the tf32 operand, K-major without
+            // swizzle: core matrices of 8 channels x 16 bytes, 8-channel
+            // groups 256 bytes apart and the two k-groups 128 bytes apart (so
+            // every access of the product stays inside the 4 KB tile);
+            // channel c's row is (v, 0, 0, 0) in both k-groups; 4 channels
+            // per lane
+            const float sinv = ldexpf(1.0f, -__ldg(&P.vexp[bh]));
+            const float4 u = __ldg(reinterpret_cast<const float4*>(
+                P.vmean + (static_cast<size_t>(bh) * g.nb + j) * D + lane * 4));
+            const float uv[4] = {u.x * sinv, u.y * sinv, u.z * sinv, u.w * sinv};
+            unsigned char* mt = sMT + s * C::MT_BYTES;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int c = lane * 4 + q;
+              const int off = (c >> 3) * 256 + (c & 7) * 16;
+              const float4 row = make_float4(uv[q], 0.f, 0.f, 0.f);
+              *reinterpret_cast<float4*>(mt + off) = row;
+              *reinterpret_cast<float4*>(mt + 128 + off) = row;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
         if (lane == 0) {
           if (LB && isv) {
             // E4M3 codes of block j, [d][bs] bytes: one 128-byte-wide box
@@ -457,6 +488,11 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
               const uint64_t bd = smem_desc_sw128(v_addr + kk * 32, 16, 1024);
               mma_ts_f8(tmem + C::COL_O, aP + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
             }
+            // V-Smooth's mean term: O += [l0 0 0 0 l1 0 0 0] . [mu/2^e rows],
+            // A = the groups' partial row sums in columns 32..39 of the S buffer
+            const uint32_t mt_addr = smem_u32(sMT + s * C::MT_BYTES);
+            mma_ts_tf32(tmem + C::COL_O, aP + 32, smem_desc_noswizzle(mt_addr, 128, 256),
+                        C::IDESC_MEAN, 1u);
           } else {
             const uint32_t v_addr = smem_u32(sV + s * C::TILE_BYTES);
 #pragma unroll
@@ -657,9 +693,9 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           if constexpr (LB) {
             // E4M3 codes (4 per column) over this group's quarter of S
             tmem_st16(scol + wg * (CPW / 4), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-            // this block's partial row sum and the reference it is relative to
-            reinterpret_cast<float2*>(P.lsum)[((static_cast<size_t>(blockIdx.x * 2 + (ouses & 1)) * g.nb + i) * 2 + wg) * 128 + t] =
-                make_float2(lblk, m);
+            // this group's share of the block's row sum: k = 4 * group of
+            // the tf32 mean product's A operand (columns 32..39)
+            tmem_st4(scol + 32 + wg * 4, __float_as_uint(lblk), 0u, 0u, 0u);
           } else if constexpr (CPW >= 64) {
             // P (bf16 pairs) over the first half of this group's S columns
             const uint32_t pcol = scol + wg * (CPW / 2);
@@ -698,37 +734,10 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
 #pragma unroll
         for (int k = 1; k < NWG; ++k) lt += xsum[k * 128 + t];
         if constexpr (LB) {
-          // V-Smooth: O = (2^e * P.codes + sum_j l_j mu_j) / l, with l_j the
-          // row's per-block sums of both groups
+          // O holds P.codes + sum_j l_j mu_j / 2^e: scale back by 2^e
           const float sig = ldexpf(1.0f, __ldg(&P.vexp[bh]));
-          const float2* lp = reinterpret_cast<const float2*>(P.lsum) +
-                             (static_cast<size_t>(blockIdx.x * 2 + ((ouses - 1) & 1)) * g.nb) * 256 + t;
 #pragma unroll
-          for (int half = 0; half < DPW; half += 32) {  // 32 columns at a time
-            float mt[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) mt[c] = 0.f;
-            for (int q = 0; q < n; ++q) {
-              int j = __ldg(&P.col_idx[start + q]);
-              j = (j < 0 || j >= g.nb) ? 0 : j;
-              // both groups' partial sums, brought to the final reference
-              const float2 p0 = lp[q * 256], p1 = lp[q * 256 + 128];
-              const float lj = (p0.x + p1.x) * ex2_approx(p0.y - m);
-              const float4* mu = reinterpret_cast<const float4*>(
-                  P.vmean + (static_cast<size_t>(bh) * g.nb + j) * D + wg * DPW + half);
-#pragma unroll
-              for (int c4 = 0; c4 < 8; ++c4) {
-                const float4 u = __ldg(&mu[c4]);
-                mt[4 * c4 + 0] = fmaf(lj, u.x, mt[4 * c4 + 0]);
-                mt[4 * c4 + 1] = fmaf(lj, u.y, mt[4 * c4 + 1]);
-                mt[4 * c4 + 2] = fmaf(lj, u.z, mt[4 * c4 + 2]);
-                mt[4 * c4 + 3] = fmaf(lj, u.w, mt[4 * c4 + 3]);
-              }
-            }
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              orr[half + c] = __float_as_uint(fmaf(sig, __uint_as_float(orr[half + c]), mt[c]));
-          }
+          for (int c = 0; c < DPW; ++c) orr[c] = __float_as_uint(sig * __uint_as_float(orr[c]));
         }
         if (t < BS) {
           const float inv = qvalid ? 1.0f / lt : 0.f;
@@ -991,7 +1000,6 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
   ap.scale_log2 = scale_log2;
   ap.vmean = nullptr;
   ap.vexp = nullptr;
-  ap.lsum = nullptr;
   if (g.d == 128 && g.bs == 128) return launch_tc<128, 128>(p, qt, kt, vt, ap, st);
   if (g.d == 128 && g.bs == 64) return launch_tc<128, 64>(p, qt, kt, vt, ap, st);
   if (g.d == 64 && g.bs == 128) return launch_tc<64, 128>(p, qt, kt, vt, ap, st);
@@ -999,16 +1007,10 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
   return cudaErrorInvalidValue;
 }
 
-size_t lowbit_scratch_bytes(const sba_plan* p, int sms) {
-  return static_cast<size_t>(std::max(1, std::min(sms, p->info.rows))) * 2 * p->info.nb * 2 * 128 *
-         sizeof(float2);
-}
-
 cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const void* kt, const void* vq,
                                     const float* vmean, const int32_t* vexp, const int32_t* row_ptr,
                                     const int32_t* col_idx, const int32_t* work_order, void* ot,
-                                    float* lse, uint64_t* trace, float* lsum, void* workspace,
-                                    cudaStream_t st) {
+                                    float* lse, uint64_t* trace, void* workspace, cudaStream_t st) {
   KGeom g = make_kgeom(p);
   AttnParams ap;
   ap.g = g;
@@ -1025,7 +1027,6 @@ cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const voi
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(g.d)));
   ap.vmean = vmean;
   ap.vexp = vexp;
-  ap.lsum = lsum;
   if (g.d == 128 && g.bs == 128) return launch_tc<128, 128, true>(p, qt, kt, vq, ap, st);
   return cudaErrorInvalidValue;
 }

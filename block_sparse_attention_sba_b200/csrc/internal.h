@@ -86,11 +86,7 @@ cudaError_t launch_smooth_v(const sba_plan* p, const void* vt, void* vq, float* 
 cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const void* kt, const void* vq,
                                     const float* vmean, const int32_t* vexp, const int32_t* row_ptr,
                                     const int32_t* col_idx, const int32_t* work_order, void* ot,
-                                    float* lse, uint64_t* trace, float* lsum, void* workspace,
-                                    cudaStream_t st);
-// Bytes of per-block row-sum scratch the low-bit attention needs on a GPU
-// with `sms` multiprocessors.
-size_t lowbit_scratch_bytes(const sba_plan* p, int sms);
+                                    float* lse, uint64_t* trace, void* workspace, cudaStream_t st);
 
 // Set by launch_attention when it fails before a launch for a reason that is
 // not a CUDA error (e.g. the tensor-map encoder is unavailable).

@@ -253,11 +253,6 @@ SBA_API sba_status sba_build_stripe_mask(const sba_plan* plan, const sba_stripe*
 SBA_API sba_status sba_smooth_v(const sba_plan* plan, const void* vt, void* vq, float* vmean,
                                 int32_t* vexp, void* workspace, void* stream);
 
-/* Bytes of scratch sba_attention_lowbit needs on the current device:
- * min(SMs, R) * 2 * nb * 2 * 128 * 8 (per persistent CTA and two rows: per
- * block and softmax column group, a partial row sum and its reference). */
-SBA_API sba_status sba_lowbit_scratch_bytes(const sba_plan* plan, size_t* bytes);
-
 /* Block-sparse attention with ExpCast-FP8 probabilities and V-Smooth values.
  * Per row (query block i) and selected key block j, on real keys:
  *   x = q.k / sqrt(d) * log2(e) - m, with m the row's reference maximum: the
@@ -271,7 +266,7 @@ SBA_API sba_status sba_lowbit_scratch_bytes(const sba_plan* plan, size_t* bytes)
  * Rows without blocks give o = 0 and lse = -inf; padding query slots 0.
  * Inputs as for sba_attention with vq, vmean, vexp from sba_smooth_v; the
  * longest-first persistent scheduler is always used (work_order required).
- * scratch: device, at least sba_lowbit_scratch_bytes (16-byte aligned).
+ * The block-mean term is accumulated in tensor memory; no scratch is needed.
  * bf16 plans with d = 128 and bs = 128 only (else SBA_ERR_UNSUPPORTED).
  * Results are not bit-identical to the bf16 path: E4M3 values carry ~3
  * mantissa bits, so the output departs from exact attention by a few
@@ -280,8 +275,7 @@ SBA_API sba_status sba_attention_lowbit(const sba_plan* plan, const void* qt, co
                                         const void* vq, const float* vmean, const int32_t* vexp,
                                         const int32_t* row_ptr, const int32_t* col_idx,
                                         const int32_t* work_order, void* ot, float* lse,
-                                        uint64_t* trace, void* scratch, size_t scratch_bytes,
-                                        void* workspace, void* stream);
+                                        uint64_t* trace, void* workspace, void* stream);
 
 /* Block-sparse attention forward (FVAttn abstract: attention over the
  * materialised mask). For every real query slot q of block i:

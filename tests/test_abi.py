@@ -188,16 +188,16 @@ def test_lowbit_calls_validate_before_any_launch(sba):
     plan64 = sba.Plan(1, 2, 8, 16, 16, 64, (4, 4, 4), "bf16")
     with pytest.raises(sba.SbaError) as e:
         sba.sba_attention_lowbit(plan64.handle, fake, fake, fake, fake, fake, fake, fake, fake,
-                                 fake, None, None, fake, 1 << 30, fake, stream=0)
+                                 fake, None, None, fake, stream=0)
     assert e.value.status == sba.SBA_ERR_UNSUPPORTED
     plan = sba.Plan(1, 2, 5, 20, 19, 128, (2, 8, 8), "bf16")
     with pytest.raises(sba.SbaError) as e:
         sba.sba_attention_lowbit(plan.handle, fake, fake, fake, fake, fake, fake, fake, None,
-                                 fake, None, None, fake, 1 << 30, fake, stream=0)
+                                 fake, None, None, fake, stream=0)
     assert e.value.status == sba.SBA_ERR_INVALID_ARG  # work_order is required
     with pytest.raises(sba.SbaError) as e:
         sba.sba_attention_lowbit(plan.handle, fake, fake, fake + 8, fake, fake, fake, fake, fake,
-                                 fake, None, None, fake, 1 << 30, fake, stream=0)
+                                 fake, None, None, fake, stream=0)
     assert e.value.status == sba.SBA_ERR_INVALID_ARG  # misaligned codes
     planf = sba.Plan(1, 2, 4, 8, 8, 64, (4, 4, 4), "f32")
     with pytest.raises(sba.SbaError) as e:

@@ -132,15 +132,8 @@ def test_lowbit_empty_rows_and_rejected_shapes():
     vmean = torch.empty(1, wl.H, g.nb, wl.d, dtype=torch.float32, device=dev)
     vexp = torch.empty(1, wl.H, dtype=torch.int32, device=dev)
     sba.sba_smooth_v(h, sa.vt, vq, vmean, vexp, sa.workspace)
-    nbytes = sba.sba_lowbit_scratch_bytes(h)
-    scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    with pytest.raises(sba.SbaError) as err:
-        sba.sba_attention_lowbit(h, sa.qt, sa.kt, vq, vmean, vexp, sa.row_ptr, sa.col_idx,
-                                 sa.work_order, sa.ot, sa.lse, None, scratch, nbytes - 16,
-                                 sa.workspace)
-    assert err.value.status == sba.SBA_ERR_CAPACITY
     sba.sba_attention_lowbit(h, sa.qt, sa.kt, vq, vmean, vexp, sa.row_ptr, sa.col_idx,
-                             sa.work_order, sa.ot, sa.lse, None, scratch, nbytes, sa.workspace)
+                             sa.work_order, sa.ot, sa.lse, None, sa.workspace)
     torch.cuda.synchronize()
     assert sa.check() == 0
     valid = oracle.slot_valid(g)
@@ -152,6 +145,5 @@ def test_lowbit_empty_rows_and_rejected_shapes():
     plan64 = sba.Plan(1, 2, 8, 16, 16, 64, (4, 4, 4), "bf16")
     with pytest.raises(sba.SbaError) as err:
         sba.sba_attention_lowbit(plan64.handle, sa.qt, sa.kt, vq, vmean, vexp, sa.row_ptr,
-                                 sa.col_idx, sa.work_order, sa.ot, sa.lse, None, scratch, nbytes,
-                                 sa.workspace)
+                                 sa.col_idx, sa.work_order, sa.ot, sa.lse, None, sa.workspace)
     assert err.value.status == sba.SBA_ERR_UNSUPPORTED
