@@ -147,3 +147,17 @@ def test_lowbit_empty_rows_and_rejected_shapes():
         sba.sba_attention_lowbit(plan64.handle, sa.qt, sa.kt, vq, vmean, vexp, sa.row_ptr,
                                  sa.col_idx, sa.work_order, sa.ot, sa.lse, None, sa.workspace)
     assert err.value.status == sba.SBA_ERR_UNSUPPORTED
+
+
+def test_lowbit_hilbert_order_every_row():
+    """Hilbert-ordered blocks (a partial last block): smoothing counts only the
+    real tokens of the tail block, attention masks its padding keys."""
+    _need_gpu()
+    wl = datagen.with_order(SMALL, "hilbert")
+    gpu = _run(wl)
+    assert gpu["status"] == 0
+    codes, mu, e = _check_smooth(wl, gpu)
+    g = geom_of(wl)
+    assert g.N % g.bs != 0  # the last block is partial
+    blocks = [(0, h, i) for h in range(wl.H) for i in range(g.nb)]
+    _check_attention(wl, gpu, codes, mu, e, blocks)
