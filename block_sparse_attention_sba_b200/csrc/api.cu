@@ -398,8 +398,11 @@ sba_status sba_perm_export(const sba_plan* plan, int32_t* slot_of_token) {
   for (int t = 0; t < G.T; ++t)
     for (int h = 0; h < G.Hh; ++h)
       for (int w = 0; w < G.W; ++w, ++n) {
-        const int blk = ((t / G.ct) * nH + h / G.ch) * nW + w / G.cw;
-        const int off = ((t % G.ct) * G.ch + h % G.ch) * G.cw + w % G.cw;
+        const int th = h / G.ch, tw = w / G.cw;
+        const int blk = ((t / G.ct) * nH + th) * nW + tw;
+        // rank inside the cube's real sub-box (vh x vw in h and w)
+        const int vh = std::min(G.ch, G.Hh - th * G.ch), vw = std::min(G.cw, G.W - tw * G.cw);
+        const int off = ((t % G.ct) * vh + h % G.ch) * vw + w % G.cw;
         slot_of_token[n] = blk * bs + off;
       }
   return SBA_OK;

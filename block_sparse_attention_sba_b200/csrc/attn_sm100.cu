@@ -34,7 +34,8 @@
 // Rescaling of O is skipped while the running row max grows by less than
 // 2^24 (the final normalisation uses the same reference max, so the result is
 // exact up to rounding; bf16 P up to 2^24 stays far inside fp32 range for O
-// and the row sum); padding keys of edge cubes are masked to -inf.
+// and the row sum); padding keys (the tail of a partial block) are masked to
+// -inf.
 // Low-bit variant (LB, VC-Attention abstract): E4M3 probability codes from
 // one multiply-add (ExpCast-FP8), O += P.V as an 8-bit tensor-core product
 // on V-Smooth codes, and the block-mean term sum_j l_j mu_j added to O by a
@@ -142,17 +143,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
   return mbar_wait(bar, parity, budget_ns, &never, status);
 }
 
-// Validity class of block j: cube order, bit 2 / 1 / 0 = last cube along
-// t / h / w; Hilbert order, 1 for a partial last block, else 0.
-__device__ __forceinline__ int block_type(const KGeom& g, int j) {
-  if (g.order == SBA_ORDER_HILBERT) return (j == g.nb - 1 && g.tail < g.bs) ? 1 : 0;
-  uint32_t rest, tw, tt, th;
-  g.dv_nW.divmod(static_cast<uint32_t>(j), rest, tw);
-  g.dv_nH.divmod(rest, tt, th);
-  return ((static_cast<int>(tt) == g.nT - 1) << 2) | ((static_cast<int>(th) == g.nH - 1) << 1) |
-         (static_cast<int>(tw) == g.nW - 1);
-}
-
 template <int D, int BS, bool LB>
 __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -170,8 +160,6 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 516);
   int* ring = reinterpret_cast<int*>(ctl + 528);             // [2][4]
-  uint32_t* emask = reinterpret_cast<uint32_t*>(ctl + 576);  // [8][4]
-  int* efull = reinterpret_cast<int*>(ctl + 704);            // [8]
   float* xmax = reinterpret_cast<float*>(ctl + 1024);        // [NSB][NWG][128] partial row maxima
   float* xsum = xmax + C::NSB * C::NWG * 128;                // [NWG][128] partial row sums
 
@@ -208,24 +196,6 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
     mbar_init(bar(C::B_L), C::NWG * 4);
     *abort_flag = 0;
     fence_barrier_init();
-  }
-  if (threadIdx.x >= 32 && threadIdx.x < 40) {
-    // validity masks of the 8 edge-cube types (bit 2: last in t, 1: in h, 0: in w)
-    const int ty = static_cast<int>(threadIdx.x) - 32;
-    const int vt = (ty & 4) ? g.T - (g.nT - 1) * g.ct : g.ct;
-    const int vh = (ty & 2) ? g.Hh - (g.nH - 1) * g.ch : g.ch;
-    const int vw = (ty & 1) ? g.W - (g.nW - 1) * g.cw : g.cw;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    int full = 1;
-    for (int c = 0; c < BS; ++c) {
-      const int lt = c / (g.ch * g.cw), lh = (c / g.cw) % g.ch, lw = c % g.cw;
-      const bool ok = (g.order == SBA_ORDER_HILBERT) ? (ty != 1 || c < g.tail)
-                                                    : (lt < vt && lh < vh && lw < vw);
-      if (ok) w[c >> 5] |= 1u << (c & 31);
-      else full = 0;
-    }
-    for (int k = 0; k < 4; ++k) emask[ty * 4 + k] = w[k];
-    efull[ty] = full;
   }
   if (warp == C::WARP_SISS) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -542,8 +512,8 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       const uint64_t t_start = globaltimer_ns();
       uint32_t bh, iq;
       g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
-      const int qtype = block_type(g, static_cast<int>(iq));
-      const bool qvalid = (t < BS) && ((emask[qtype * 4 + (t >> 5)] >> (t & 31)) & 1u);
+      // a block's real slots are its first block_len slots
+      const bool qvalid = t < block_len(g, static_cast<int>(iq));
       const int64_t orow = static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(iq) * BS + t;
       __nv_bfloat16* optr = P.ot + orow * D + wg * DPW;
       if (n == 0) {
@@ -572,15 +542,12 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           float s[CPW];
 #pragma unroll
           for (int e = 0; e < CPW; ++e) s[e] = __uint_as_float(sr[e]);
-          const int kt = block_type(g, j);
-          if (!efull[kt]) {
+          const int klen = block_len(g, j);
+          if (klen < BS) {
+            // padding keys (slots klen .. BS-1) are masked
 #pragma unroll
-            for (int c = 0; c < CPW / 32; ++c) {
-              const uint32_t w = emask[kt * 4 + (wg * CPW) / 32 + c];
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (!((w >> e) & 1u)) s[c * 32 + e] = -INFINITY;
-            }
+            for (int e = 0; e < CPW; ++e)
+              if (wg * CPW + e >= klen) s[e] = -INFINITY;
           }
           // partial row max over this group's columns (independent chains)
           float mc[4];
@@ -800,19 +767,8 @@ __global__ void __launch_bounds__(128)
   g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
   const int64_t head = static_cast<int64_t>(bh) * g.Npad;
 
-  auto valid_slot = [&](int blk, int c) -> bool {
-    if (g.order == SBA_ORDER_HILBERT) return blk * BS + c < g.N;
-    uint32_t rest, tw, tt, th;
-    g.dv_nW.divmod(static_cast<uint32_t>(blk), rest, tw);
-    g.dv_nH.divmod(rest, tt, th);
-    uint32_t lt, r2, lh, lw;
-    g.dv_chcw.divmod(static_cast<uint32_t>(c), lt, r2);
-    g.dv_cw.divmod(r2, lh, lw);
-    return (static_cast<int>(tt * g.ct + lt) < g.T) && (static_cast<int>(th * g.ch + lh) < g.Hh) &&
-           (static_cast<int>(tw * g.cw + lw) < g.W);
-  };
   const bool active = t < BS;
-  const bool qvalid = active && valid_slot(static_cast<int>(iq), t);
+  const bool qvalid = active && t < block_len(g, static_cast<int>(iq));
   const int64_t qrow = head + static_cast<int64_t>(iq) * BS + t;
   float q[D], o[D];
 #pragma unroll
@@ -842,8 +798,8 @@ __global__ void __launch_bounds__(128)
     }
     __syncthreads();
     if (!active) continue;
-    for (int c = 0; c < BS; ++c) {
-      if (!valid_slot(j, c)) continue;
+    const int klen = block_len(g, j);
+    for (int c = 0; c < klen; ++c) {
       float s = 0.f;
 #pragma unroll
       for (int x = 0; x < D; ++x) s = fmaf(q[x], Ks[c * (D + 1) + x], s);

@@ -65,6 +65,28 @@ struct KGeom {
 
 KGeom make_kgeom(const sba_plan* p);
 
+// Real-token extents of cube block j (cube order): the cube's sub-box inside
+// the grid.
+__device__ __forceinline__ void cube_extents(const KGeom& g, int j, int& vt, int& vh, int& vw) {
+  uint32_t rest, tw, tt, th;
+  g.dv_nW.divmod(static_cast<uint32_t>(j), rest, tw);
+  g.dv_nH.divmod(rest, tt, th);
+  vt = min(g.ct, g.T - static_cast<int>(tt) * g.ct);
+  vh = min(g.ch, g.Hh - static_cast<int>(th) * g.ch);
+  vw = min(g.cw, g.W - static_cast<int>(tw) * g.cw);
+}
+
+// Number of real tokens of block j. In both orders they occupy the block's
+// first slots (cube order: row-major over the cube's real sub-box; Hilbert
+// order: only the last block is partial), so slot o of block j is real iff
+// o < block_len(g, j).
+__device__ __forceinline__ int block_len(const KGeom& g, int j) {
+  if (g.order == SBA_ORDER_HILBERT) return j == g.nb - 1 ? g.tail : g.bs;
+  int vt, vh, vw;
+  cube_extents(g, j, vt, vh, vw);
+  return vt * vh * vw;
+}
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_reorder(const sba_plan* p, int direction, const void* src[3], void* dst[3],
                            const int32_t* token_of_slot, cudaStream_t st);

@@ -23,18 +23,9 @@ namespace {
 
 constexpr int kSmoothThreads = 128;  // one thread per channel (d <= 128)
 
-// Real-token test of slot o of block j (cube or Hilbert order).
-__device__ __forceinline__ bool slot_real(const KGeom& g, int j, int o) {
-  if (g.order == SBA_ORDER_HILBERT) return j < g.nb - 1 || o < g.tail;
-  uint32_t rest, tw, tt, th;
-  g.dv_nW.divmod(static_cast<uint32_t>(j), rest, tw);
-  g.dv_nH.divmod(rest, tt, th);
-  uint32_t lt, r2, lh, lw;
-  g.dv_chcw.divmod(static_cast<uint32_t>(o), lt, r2);
-  g.dv_cw.divmod(r2, lh, lw);
-  return static_cast<int>(tt * g.ct + lt) < g.T && static_cast<int>(th * g.ch + lh) < g.Hh &&
-         static_cast<int>(tw * g.cw + lw) < g.W;
-}
+// Real-token test of slot o of block j (cube or Hilbert order): the real
+// tokens are the block's first block_len slots.
+__device__ __forceinline__ bool slot_real(const KGeom& g, int j, int o) { return o < block_len(g, j); }
 
 // grid (nb, B*H): mu_j (fp32) and max |V - mu_j| over the block's real slots.
 __global__ void __launch_bounds__(kSmoothThreads)

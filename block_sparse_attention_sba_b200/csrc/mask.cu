@@ -67,40 +67,15 @@ __global__ void __launch_bounds__(kPoolThreads)
   const int c = threadIdx.x % vpr;
   const int rg = threadIdx.x / vpr;
 
-  int vt = g.ct, vh = g.ch, vw = g.cw, len;
-  bool full;
-  if (g.order == SBA_ORDER_HILBERT) {
-    // runs along the curve: only the last block is partial (a prefix)
-    len = (j == g.nb - 1) ? g.tail : g.bs;
-    full = len == g.bs;
-  } else {
-    uint32_t rest, tw, tt, th;
-    g.dv_nW.divmod(static_cast<uint32_t>(j), rest, tw);
-    g.dv_nH.divmod(rest, tt, th);
-    vt = min(g.ct, g.T - static_cast<int>(tt) * g.ct);
-    vh = min(g.ch, g.Hh - static_cast<int>(th) * g.ch);
-    vw = min(g.cw, g.W - static_cast<int>(tw) * g.cw);
-    full = (vt == g.ct) && (vh == g.ch) && (vw == g.cw);
-    len = vt * vh * vw;
-  }
+  // the block's real tokens occupy its first len slots (both orders)
+  const int len = block_len(g, j);
 
   const int64_t row_bytes = static_cast<int64_t>(g.d) * sizeof(T);
   const char* base = src + (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * row_bytes;
   float acc[EPV];
 #pragma unroll
   for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
-  for (int o = rg; o < g.bs; o += groups) {
-    if (!full) {
-      if (g.order == SBA_ORDER_HILBERT) {
-        if (o >= len) continue;
-      } else {
-        uint32_t lt, r2, lh, lw;
-        g.dv_chcw.divmod(static_cast<uint32_t>(o), lt, r2);
-        g.dv_cw.divmod(r2, lh, lw);
-        if (static_cast<int>(lt) >= vt || static_cast<int>(lh) >= vh || static_cast<int>(lw) >= vw)
-          continue;
-      }
-    }
+  for (int o = rg; o < len; o += groups) {
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + o * row_bytes + c * 16));
     accum_vec<T>(acc, v);
   }

@@ -6,10 +6,12 @@
 //
 // One CTA moves one cube of one (tensor, b, h): bs rows of d elements, as
 // 16-byte vectors. Cube-order rows are contiguous (bs*d*esize bytes per cube)
-// and raster rows of one cube line (cw consecutive w) are contiguous too, so
-// both sides stream in long coalesced runs. Pure bit copy; padding slots are
-// written as zeros (reorder) or skipped (unreorder). HBM-bound: every byte is
-// read once and written once.
+// and raster rows of one cube line (the cube's consecutive w) are contiguous
+// too, so both sides stream in long coalesced runs. Inside an edge cube the
+// real tokens take the first slots, row-major over the cube's real sub-box,
+// and padding the tail. Pure bit copy; padding slots are written as zeros
+// (reorder) or skipped (unreorder). HBM-bound: every byte is read once and
+// written once.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -41,6 +43,10 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(KGeom g, ReorderArgs 
   g.dv_nW.divmod(static_cast<uint32_t>(j), rest, tw);
   g.dv_nH.divmod(rest, tt, th);
   const int t0 = tt * g.ct, h0 = th * g.ch, w0 = tw * g.cw;
+  // real sub-box of this cube; its tokens fill slots [0, len) row-major
+  const int vh = min(g.ch, g.Hh - h0), vw = min(g.cw, g.W - w0);
+  const int len = min(g.ct, g.T - t0) * vh * vw;
+  const bool full = len == g.bs;
 
   const int64_t row_bytes = static_cast<int64_t>(g.d) * esize;
   const int64_t packed_base = (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * row_bytes;
@@ -67,12 +73,25 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(KGeom g, ReorderArgs 
       valid = tok >= 0;
       n = tok;
     } else {
-      uint32_t lt, r2, lh, lw;
-      g.dv_chcw.divmod(static_cast<uint32_t>(o), lt, r2);
-      g.dv_cw.divmod(r2, lh, lw);
-      const int t = t0 + lt, hh = h0 + lh, w = w0 + lw;
-      valid = (t < g.T) && (hh < g.Hh) && (w < g.W);
-      n = (static_cast<int64_t>(t) * g.Hh + hh) * g.W + w;
+      int lt, lh, lw;
+      if (full) {
+        uint32_t a, r2, b, c;
+        g.dv_chcw.divmod(static_cast<uint32_t>(o), a, r2);
+        g.dv_cw.divmod(r2, b, c);
+        lt = static_cast<int>(a);
+        lh = static_cast<int>(b);
+        lw = static_cast<int>(c);
+      } else {
+        // edge cube: rank o among the real sub-box's tokens (plain division;
+        // only the edge cubes of the grid take this branch)
+        const int area = vh * vw;
+        lt = o / area;
+        const int r2 = o - lt * area;
+        lh = r2 / vw;
+        lw = r2 - lh * vw;
+      }
+      valid = o < len;
+      n = (static_cast<int64_t>(t0 + lt) * g.Hh + (h0 + lh)) * g.W + (w0 + lw);
     }
     const int64_t raster = raster_base + n * sN_bytes + c * 16;
     const int64_t packed = packed_base + static_cast<int64_t>(o) * row_bytes + c * 16;

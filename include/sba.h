@@ -23,13 +23,16 @@
  *   of ct x ch x cw tokens; every cube is one block of bs = ct*ch*cw slots.
  *   The cube grid is nT x nH x nW with nT = ceil(T/ct) etc., nb = nT*nH*nW
  *   blocks per head and Npad = nb*bs slots per head. A grid that does not
- *   divide into whole cubes is padded: padding slots keep their geometric
- *   place inside their cube, hold zeros after sba_reorder, are never attended
- *   to as keys and produce zero output rows.
- * - Token order: raster token n = (t*Hh + h)*W + w. Slot of a token:
- *   blk*bs + ((t%ct)*ch + h%ch)*cw + w%cw with
- *   blk = ((t/ct)*nH + h/ch)*nW + w/cw (cubes row-major over the cube grid,
- *   tokens row-major inside a cube).
+ *   divide into whole cubes is padded: an edge cube's real tokens take its
+ *   first slots and padding the rest, so the real slots of every block are a
+ *   prefix of it. Padding slots hold zeros after sba_reorder, are never
+ *   attended to as keys and produce zero output rows.
+ * - Token order: raster token n = (t*Hh + h)*W + w lies in cube
+ *   blk = ((t/ct)*nH + h/ch)*nW + w/cw (cubes row-major over the cube grid).
+ *   With the cube's real extents vh = min(ch, Hh - (h/ch)*ch) and
+ *   vw = min(cw, W - (w/cw)*cw), its slot is
+ *   blk*bs + ((t%ct)*vh + h%ch)*vw + w%cw (tokens row-major inside the
+ *   cube's real sub-box; ((t%ct)*ch + h%ch)*cw + w%cw for a complete cube).
  * - Hilbert order (DFSAttn: Hilbert-curve token reordering), when the
  *   geometry's order is SBA_ORDER_HILBERT: a token's slot is its rank along a
  *   3-D Hilbert curve (Skilling's construction, axes t, h, w) over the

@@ -20,10 +20,12 @@ What it computes, step by step, and the passages each step follows:
 
 Readings where the pages are silent (each listed in the design notes):
 
-* ragged grids are padded up to whole cubes; a padding slot keeps its
-  geometric place inside its cube and holds zeros;
+* ragged grids are padded up to whole cubes; inside an edge cube the real
+  tokens come first, row-major (t, h, w) over the cube's real sub-box, and the
+  padding slots (zeros) fill the tail of the block, so every block's real
+  slots are a prefix of it;
 * cubes are ordered row-major over the cube grid (t, h, w) and tokens row-major
-  inside a cube;
+  inside a cube (for a complete cube: offset ((t%ct)*ch + h%ch)*cw + w%cw);
 * pooled means divide by the number of valid tokens of the block;
 * no length correction of partial blocks, no forced diagonal, no causality;
 * Top-p takes the shortest prefix with cumulative mass >= p (inclusive);
@@ -47,7 +49,8 @@ import numpy as np
 class Geom:
     """Grid and block geometry (FVAttn abstract: video-aware block organization).
 
-    order "cube": blocks are ct x ch x cw cubes (padding inside edge cubes).
+    order "cube": blocks are ct x ch x cw cubes (an edge cube keeps its real
+    tokens in its first slots and padding in the rest).
     order "hilbert": tokens follow a 3-D Hilbert curve over (t, h, w) and every
     run of bs = ct*ch*cw consecutive tokens is a block; only the last block
     can be partial (DFSAttn: Hilbert-curve token reordering)."""
@@ -144,8 +147,12 @@ def slot_of_token(g: Geom) -> np.ndarray:
     """Slot of every raster token ``n = (t*Hh + h)*W + w``.
 
     Hilbert order: slot = rank of the token's Hilbert index among all tokens.
-    Cube order: the token lands in cube ``blk = (t//ct * nH + h//ch) * nW + w//cw`` at
-    in-cube offset ``((t%ct)*ch + h%ch)*cw + w%cw``; slot = blk*bs + offset.
+    Cube order: the token lands in cube ``blk = (t//ct * nH + h//ch) * nW + w//cw``.
+    The cube's real sub-box has extents ``vt = min(ct, T - t//ct*ct)`` (and vh,
+    vw alike); the token's in-cube offset is ``((t%ct)*vh + h%ch)*vw + w%cw``,
+    its rank row-major over that sub-box, so the real tokens of a block fill
+    slots ``[0, vt*vh*vw)`` and padding the rest; slot = blk*bs + offset.
+    For a complete cube this is ``((t%ct)*ch + h%ch)*cw + w%cw``.
     """
     if g.order == "hilbert":
         # the token's rank along the curve among the grid's tokens
@@ -157,26 +164,32 @@ def slot_of_token(g: Geom) -> np.ndarray:
         return slot
     t, h, w = np.meshgrid(np.arange(g.T), np.arange(g.Hh), np.arange(g.W), indexing="ij")
     t, h, w = t.ravel(), h.ravel(), w.ravel()
-    blk = ((t // g.ct) * g.nH + (h // g.ch)) * g.nW + (w // g.cw)
-    off = ((t % g.ct) * g.ch + (h % g.ch)) * g.cw + (w % g.cw)
+    th, tw = h // g.ch, w // g.cw
+    blk = ((t // g.ct) * g.nH + th) * g.nW + tw
+    vh = np.minimum(g.ch, g.Hh - th * g.ch)   # real extents of the token's cube
+    vw = np.minimum(g.cw, g.W - tw * g.cw)
+    off = ((t % g.ct) * vh + (h % g.ch)) * vw + (w % g.cw)
     return (blk * g.bs + off).astype(np.int64)
 
 
 def slot_of_token_loops(g: Geom) -> np.ndarray:
     """The same permutation written as explicit loops over cubes and in-cube
-    positions (small grids only): enumerate slots in order, skip padding."""
+    positions (small grids only): inside every cube, hand out its first slots
+    to the real tokens in row-major (t, h, w) order; the rest is padding."""
     out = np.full(g.N, -1, dtype=np.int64)
-    s = 0
+    blk = 0
     for tt in range(g.nT):
         for th in range(g.nH):
             for tw in range(g.nW):
+                s = blk * g.bs
                 for lt in range(g.ct):
                     for lh in range(g.ch):
                         for lw in range(g.cw):
                             t, h, w = tt * g.ct + lt, th * g.ch + lh, tw * g.cw + lw
                             if t < g.T and h < g.Hh and w < g.W:
                                 out[(t * g.Hh + h) * g.W + w] = s
-                            s += 1
+                                s += 1
+                blk += 1
     return out
 
 

@@ -70,6 +70,11 @@ def test_perm_is_injective_onto_valid_slots_and_cubes_are_boxes(g):
         m = blk == b
         for c, e in ((t[m], g.ct), (h[m], g.ch), (w[m], g.cw)):
             assert c.min() // e == c.max() // e  # one aligned box per block
+    # the real slots of every block are a prefix of it (padding at the tail)
+    V = valid.reshape(g.nb, g.bs)
+    for b in range(g.nb):
+        n_real = int(V[b].sum())
+        assert V[b, :n_real].all() and not V[b, n_real:].any()
     # closed form for block lengths: product of per-axis clipped extents
     L = oracle.block_len(g).reshape(g.nT, g.nH, g.nW)
     for tt, th, tw in itertools.product(range(g.nT), range(g.nH), range(g.nW)):
