@@ -42,7 +42,7 @@ EXPORTED = ["sba_plan_create", "sba_plan_destroy", "sba_plan_query", "sba_worksp
             "sba_check_device_status", "sba_debug_timeout_probe", "sba_perm_export",
             "sba_attention_grid_size", "sba_status_string", "sba_last_error",
             "sba_build_mask_noalloc", "sba_build_stripe_mask", "sba_smooth_v",
-            "sba_attention_lowbit"]
+            "sba_attention_lowbit", "sba_noalloc_status"]
 
 
 class sba_geometry(ctypes.Structure):
@@ -84,6 +84,7 @@ _sig = {
     "sba_smooth_v": [_vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "sba_attention_lowbit": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "sba_check_device_status": [_vp, _vp, _vp],
+    "sba_noalloc_status": [_vp],
     "sba_debug_timeout_probe": [_vp, _vp, ctypes.c_uint64, _vp],
     "sba_perm_export": [_vp, ctypes.POINTER(ctypes.c_int32)],
     "sba_attention_grid_size": [],
@@ -133,13 +134,18 @@ def _stream(stream) -> Optional[int]:
 
 # ----------------------------------------------------------------- raw C ABI
 
+_plan_heads = {}  # plan handle -> H (the C side reads top_p[0..H-1])
+
+
 def sba_plan_create(geom: sba_geometry) -> int:
     h = _vp()
     _check(_lib.sba_plan_create(ctypes.byref(geom), ctypes.byref(h)), "sba_plan_create")
+    _plan_heads[h.value] = int(geom.H)
     return h.value
 
 
 def sba_plan_destroy(plan: int) -> None:
+    _plan_heads.pop(plan, None)
     _lib.sba_plan_destroy(plan)
 
 
@@ -163,9 +169,20 @@ def sba_unreorder(plan: int, ot, o, workspace=None, stream=None) -> None:
            "sba_unreorder")
 
 
+def _top_p_array(plan: int, top_p: Sequence[float]):
+    """ctypes float array of one Top-p value per head (the C side reads H of
+    them, so a shorter sequence is refused here instead of read past)."""
+    H = _plan_heads.get(plan)
+    if H is None:
+        raise ValueError("unknown plan handle (create plans with sba_plan_create)")
+    if len(top_p) != H:
+        raise ValueError(f"top_p has {len(top_p)} values; the plan has H = {H} heads")
+    return (ctypes.c_float * H)(*[float(x) for x in top_p])
+
+
 def sba_build_mask(plan: int, qt, kt, top_p: Sequence[float], top_k: int, bitmask, row_cnt,
                    row_ptr, col_idx, work_order, workspace, stream=None) -> None:
-    arr = (ctypes.c_float * len(top_p))(*[float(x) for x in top_p])
+    arr = _top_p_array(plan, top_p)
     _check(_lib.sba_build_mask(plan, _ptr(qt), _ptr(kt), arr, int(top_k), _ptr(bitmask),
                                _ptr(row_cnt), _ptr(row_ptr), _ptr(col_idx), _ptr(work_order),
                                _ptr(workspace), _stream(stream)), "sba_build_mask")
@@ -175,7 +192,7 @@ def sba_build_mask_noalloc(plan: int, qt, kt, top_p: Sequence[float], top_k: int
                            row_cnt, row_ptr, col_idx, work_order, stream=None) -> None:
     """sba_build_mask without a workspace: the library's static scratch is used
     instead (see include/sba.h for the size limit and the sharing rules)."""
-    arr = (ctypes.c_float * len(top_p))(*[float(x) for x in top_p])
+    arr = _top_p_array(plan, top_p)
     _check(_lib.sba_build_mask_noalloc(plan, _ptr(qt), _ptr(kt), arr, int(top_k), _ptr(bitmask),
                                        _ptr(row_cnt), _ptr(row_ptr), _ptr(col_idx),
                                        _ptr(work_order), _stream(stream)), "sba_build_mask_noalloc")
@@ -208,6 +225,12 @@ def sba_attention(plan: int, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse=N
     _check(_lib.sba_attention(plan, _ptr(qt), _ptr(kt), _ptr(vt), _ptr(row_ptr), _ptr(col_idx),
                               _ptr(work_order), _ptr(ot), _ptr(lse), int(sched), _ptr(trace),
                               _ptr(workspace), _stream(stream)), "sba_attention")
+
+
+def sba_noalloc_status(stream=None) -> int:
+    """Status of sba_build_mask_noalloc's static scratch (syncs; does not
+    raise on device-side errors)."""
+    return _lib.sba_noalloc_status(_stream(stream))
 
 
 def sba_check_device_status(plan: int, workspace, stream=None) -> int:

@@ -187,7 +187,7 @@ sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
   p->info.max_nnz = R * nb;
   p->ws_ctrl = 0;
   p->ws_qbar = 256;
-  const size_t pooled = align256(static_cast<size_t>(R) * G.d * sizeof(float));
+  const size_t pooled = align256(static_cast<size_t>(R) * G.d * sizeof(double));
   p->ws_kbar = p->ws_qbar + pooled;
   p->ws_perm = p->ws_kbar + pooled;
   p->info.workspace_bytes = p->ws_perm;
@@ -281,8 +281,12 @@ sba_status sba_build_mask(const sba_plan* plan, const void* qt, const void* kt, 
     if (!(p > 0.0f) || !(p <= 1.0f))
       return fail(SBA_ERR_INVALID_ARG, "top_p[%d] = %g; must lie in (0, 1]", h, (double)p);
   }
+  char* ws = static_cast<char*>(workspace);
   cudaError_t e = launch_build_mask(plan, qt, kt, top_p, top_k, bitmask, row_cnt, row_ptr, col_idx,
-                                    work_order, workspace, static_cast<cudaStream_t>(stream));
+                                    work_order, reinterpret_cast<double*>(ws + plan->ws_qbar),
+                                    reinterpret_cast<double*>(ws + plan->ws_kbar),
+                                    &reinterpret_cast<Ctrl*>(ws + plan->ws_ctrl)->status,
+                                    static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_build_mask launch");
 }
 

@@ -13,7 +13,7 @@ struct sba_plan {
   sba_plan_info info;
   int esize;               // bytes per element (2 or 4)
   size_t ws_ctrl;          // offset of the control block (status, counters)
-  size_t ws_qbar, ws_kbar; // offsets of the pooled means (fp32 [B*H][nb][d])
+  size_t ws_qbar, ws_kbar; // offsets of the pooled means (fp64 [B*H][nb][d])
   size_t ws_perm;          // Hilbert order: offset of token_of_slot (int32 [Npad])
   uint64_t wait_budget_ns; // bounded-wait limit for device waits
   std::vector<int32_t> slot_of_token;  // Hilbert order: int32 [N]
@@ -90,10 +90,12 @@ __device__ __forceinline__ int block_len(const KGeom& g, int j) {
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_reorder(const sba_plan* p, int direction, const void* src[3], void* dst[3],
                            const int32_t* token_of_slot, cudaStream_t st);
+// The four mask launches with their scratch given: pooled means qbar, kbar
+// (fp64 [B*H][nb][d] each) and the status word that device checks set.
 cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
                               const float* top_p, int top_k, uint32_t* bitmask, int32_t* row_cnt,
                               int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
-                              void* workspace, cudaStream_t st);
+                              double* qbar, double* kbar, uint32_t* status, cudaStream_t st);
 cudaError_t launch_build_stripe_mask(const sba_plan* p, const sba_stripe* params,
                                      uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
                                      int32_t* col_idx, int32_t* work_order, void* workspace,

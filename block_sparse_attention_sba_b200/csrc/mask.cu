@@ -33,35 +33,37 @@ namespace {
 constexpr int kPoolThreads = 256;
 
 template <typename T>
-__device__ __forceinline__ void accum_vec(float* acc, const uint4& v);
+__device__ __forceinline__ void accum_vec(double* acc, const uint4& v);
 
 template <>
-__device__ __forceinline__ void accum_vec<__nv_bfloat16>(float* acc, const uint4& v) {
+__device__ __forceinline__ void accum_vec<__nv_bfloat16>(double* acc, const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += __uint_as_float(w[i] << 16);
-    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+    acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
+    acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
   }
 }
 
 template <>
-__device__ __forceinline__ void accum_vec<float>(float* acc, const uint4& v) {
-  acc[0] += __uint_as_float(v.x);
-  acc[1] += __uint_as_float(v.y);
-  acc[2] += __uint_as_float(v.z);
-  acc[3] += __uint_as_float(v.w);
+__device__ __forceinline__ void accum_vec<float>(double* acc, const uint4& v) {
+  acc[0] += static_cast<double>(__uint_as_float(v.x));
+  acc[1] += static_cast<double>(__uint_as_float(v.y));
+  acc[2] += static_cast<double>(__uint_as_float(v.z));
+  acc[3] += static_cast<double>(__uint_as_float(v.w));
 }
 
-// grid (nb, B*H, 2): z = 0 pools qt, z = 1 pools kt.
+// grid (nb, B*H, 2): z = 0 pools qt, z = 1 pools kt. Sums in fp64 (a sum of
+// bf16 or fp32 values is exact there for any realistic spread of exponents),
+// one division by the number of real tokens.
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
     pool_kernel(KGeom g, const char* __restrict__ qt, const char* __restrict__ kt,
-                float* __restrict__ qbar, float* __restrict__ kbar) {
+                double* __restrict__ qbar, double* __restrict__ kbar) {
   constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
   const int j = blockIdx.x, bh = blockIdx.y;
   const char* src = blockIdx.z == 0 ? qt : kt;
-  float* dst = blockIdx.z == 0 ? qbar : kbar;
+  double* dst = blockIdx.z == 0 ? qbar : kbar;
   const int vpr = g.d / EPV;            // vectors per row (8..32)
   const int groups = kPoolThreads / vpr;  // row groups
   const int c = threadIdx.x % vpr;
@@ -72,178 +74,239 @@ __global__ void __launch_bounds__(kPoolThreads)
 
   const int64_t row_bytes = static_cast<int64_t>(g.d) * sizeof(T);
   const char* base = src + (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * row_bytes;
-  float acc[EPV];
+  double acc[EPV];
 #pragma unroll
-  for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
+  for (int e = 0; e < EPV; ++e) acc[e] = 0.0;
   for (int o = rg; o < len; o += groups) {
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + o * row_bytes + c * 16));
     accum_vec<T>(acc, v);
   }
-  __shared__ float red[kPoolThreads * 8];
+  __shared__ double red[kPoolThreads * 8];
   // red[rg][d]: reduce over row groups
 #pragma unroll
   for (int e = 0; e < EPV; ++e) red[rg * g.d + c * EPV + e] = acc[e];
   __syncthreads();
-  const float inv_len = 1.0f / static_cast<float>(len);
+  const double dlen = static_cast<double>(len);
   for (int col = threadIdx.x; col < g.d; col += kPoolThreads) {
-    float s = 0.f;
+    double s = 0.0;
     for (int r = 0; r < groups; ++r) s += red[r * g.d + col];
-    dst[(static_cast<int64_t>(bh) * g.nb + j) * g.d + col] = s * inv_len;
+    dst[(static_cast<int64_t>(bh) * g.nb + j) * g.d + col] = s / dlen;
   }
 }
 
 // ---------------------------------------------------------- score + select
+// All of it in fp64, so that the routing decision is the exact one except
+// where the cumulative mass at the cut lies within rounding of p.
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kRQ = 16;      // query blocks per CTA
-constexpr int kKC = 64;      // key blocks per shared-memory chunk
+constexpr int kMaxE = 32;    // probabilities per lane (nb <= 1024)
 
 struct SelectArgs {
   float top_p[256];
 };
 
-__device__ __forceinline__ unsigned long long key_of(float p, int j) {
-  return (static_cast<unsigned long long>(~__float_as_uint(p)) << 32) | static_cast<uint32_t>(j);
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
-// Ascending bitonic sort of n (power of two, >= 32) 64-bit keys by one warp.
-__device__ void warp_bitonic_sort(unsigned long long* a, int n) {
-  const int lane = threadIdx.x & 31;
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = lane; i < (n >> 1); i += 32) {
-        const int lo = 2 * jj * (i / jj) + (i % jj);
-        const int hi = lo + jj;
-        const unsigned long long x = a[lo], y = a[hi];
-        const bool up = (lo & k) == 0;
-        if ((x > y) == up) {
-          a[lo] = y;
-          a[hi] = x;
-        }
-      }
-      __syncwarp();
-    }
-  }
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
-// grid (ceil(nb/kRQ), B*H). Dynamic shared memory:
-//   qs [kRQ][d+4] f32 | S [kRQ][nkp] f32 | union{ ks [kKC][d+4] f32,
-//   sort keys [kSelWarps][nkp] u64 } | words [kSelWarps][32] u32
+// grid (ceil(nb/kRQ), B*H), kSelThreads threads. Dynamic shared memory:
+//   qs [kRQ][d] f64 | S [kRQ][nb] f64
+// Phase 1: thread t computes the scores of key blocks t, t+256, ... against
+// the CTA's kRQ query blocks (fp64 FMA, K rows streamed from L1).
+// Phase 2: one warp per query block: fp64 softmax over the key blocks, then
+// the cut: the largest probability v with mass(P >= v) >= p found by
+// bisection on the bit pattern of v (warp mass sums), the ties of v taken in
+// index order until the mass reaches p; the Top-k floor by the same
+// bisection on counts. No sort.
 __global__ void __launch_bounds__(kSelThreads)
-    select_kernel(KGeom g, const float* __restrict__ qbar, const float* __restrict__ kbar,
-                  SelectArgs sa, int top_k, int nkp, uint32_t* __restrict__ bitmask,
+    select_kernel(KGeom g, const double* __restrict__ qbar, const double* __restrict__ kbar,
+                  SelectArgs sa, int top_k, uint32_t* __restrict__ bitmask,
                   int32_t* __restrict__ row_cnt) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int d = g.d, nb = g.nb, ld = d + 4;
+  const int d = g.d, nb = g.nb;
   const int bh = blockIdx.y;
   const int q0 = blockIdx.x * kRQ;
-  float* qs = reinterpret_cast<float*>(smem);
-  float* S = qs + kRQ * ld;
-  unsigned char* uni = reinterpret_cast<unsigned char*>(S + kRQ * nkp);
-  float* ks = reinterpret_cast<float*>(uni);
-  const size_t uni_bytes = max(static_cast<size_t>(kKC) * ld * 4, static_cast<size_t>(kSelWarps) * nkp * 8);
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(uni);
-  uint32_t* wbuf = reinterpret_cast<uint32_t*>(uni + uni_bytes);
-
+  double* qs = reinterpret_cast<double*>(smem);
+  double* S = qs + kRQ * d;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float* qsrc = qbar + static_cast<int64_t>(bh) * nb * d;
-  const float* ksrc = kbar + static_cast<int64_t>(bh) * nb * d;
+  const double* qsrc = qbar + static_cast<int64_t>(bh) * nb * d;
+  const double* ksrc = kbar + static_cast<int64_t>(bh) * nb * d;
 
   // stage the query rows (zero rows past nb)
   for (int e = tid; e < kRQ * d; e += kSelThreads) {
     const int r = e / d, c = e % d;
-    qs[r * ld + c] = (q0 + r < nb) ? qsrc[static_cast<int64_t>(q0 + r) * d + c] : 0.f;
+    qs[e] = (q0 + r < nb) ? qsrc[static_cast<int64_t>(q0 + r) * d + c] : 0.0;
   }
-  const float scale = rsqrtf(static_cast<float>(d));
-  const int kk = tid % kKC;       // key within chunk
-  const int rg = tid / kKC;       // rows rg*4 .. rg*4+3
-  for (int j0 = 0; j0 < nb; j0 += kKC) {
-    __syncthreads();
-    for (int e = tid; e < kKC * (d / 4); e += kSelThreads) {
-      const int r = e / (d / 4), c4 = e % (d / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + r < nb) v = *reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j0 + r) * d + c4 * 4);
-      *reinterpret_cast<float4*>(ks + r * ld + c4 * 4) = v;
-    }
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* krow = ks + kk * ld;
-    for (int c = 0; c < d; c += 4) {
-      const float4 kv = *reinterpret_cast<const float4*>(krow + c);
+  __syncthreads();
+  const double sqrt_d = sqrt(static_cast<double>(d));
+  for (int j = tid; j < nb; j += kSelThreads) {
+    double acc[kRQ];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float4 qv = *reinterpret_cast<const float4*>(qs + (rg * 4 + r) * ld + c);
-        acc[r] = fmaf(qv.x, kv.x, acc[r]);
-        acc[r] = fmaf(qv.y, kv.y, acc[r]);
-        acc[r] = fmaf(qv.z, kv.z, acc[r]);
-        acc[r] = fmaf(qv.w, kv.w, acc[r]);
+    for (int r = 0; r < kRQ; ++r) acc[r] = 0.0;
+    const double2* krow = reinterpret_cast<const double2*>(ksrc + static_cast<int64_t>(j) * d);
+    for (int c2 = 0; c2 < d / 2; ++c2) {
+      const double2 kv = __ldg(krow + c2);
+#pragma unroll
+      for (int r = 0; r < kRQ; ++r) {
+        const double2 qv = reinterpret_cast<const double2*>(qs + r * d)[c2];
+        acc[r] = fma(qv.x, kv.x, acc[r]);
+        acc[r] = fma(qv.y, kv.y, acc[r]);
       }
     }
-    if (j0 + kk < nb) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) S[(rg * 4 + r) * nkp + j0 + kk] = acc[r] * scale;
-    }
+    for (int r = 0; r < kRQ; ++r) S[r * nb + j] = acc[r] / sqrt_d;
   }
-  __syncthreads();  // all scores written; ks area becomes sort keys
+  __syncthreads();
 
   uint32_t h;
   {
     uint32_t bq;
     g.dv_H.divmod(static_cast<uint32_t>(bh), bq, h);
   }
-  const float p = sa.top_p[h];
-  unsigned long long* kw = keys + static_cast<size_t>(warp) * nkp;
-  uint32_t* words = wbuf + warp * 32;
-  const int seg = nkp / 32;
+  const double p = static_cast<double>(sa.top_p[h]);
+  const int E = (nb + 31) >> 5;
   for (int r = warp; r < kRQ; r += kSelWarps) {
     const int i = q0 + r;
     if (i >= nb) break;
-    const float* srow = S + r * nkp;
-    float mx = -INFINITY;
-    for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, srow[j]);
+    const double* srow = S + r * nb;
+    // softmax in fp64: shift by the row max, exp, divide by the sum
+    double mx = -INFINITY;
+    for (int j = lane; j < nb; j += 32) mx = fmax(mx, srow[j]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
-    for (int j = lane; j < nb; j += 32) sum += expf(srow[j] - mx);
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    double pv[kMaxE];
+    double esum = 0.0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float inv = 1.0f / sum;
-    for (int j = lane; j < nkp; j += 32)
-      kw[j] = (j < nb) ? key_of(expf(srow[j] - mx) * inv, j) : ~0ull;
-    words[lane] = 0u;
-    __syncwarp();
-    warp_bitonic_sort(kw, nkp);
-
-    // cumulative mass along the sorted order: lane owns positions [lane*seg, +seg)
-    float local = 0.f;
-    for (int e = 0; e < seg; ++e) local += __uint_as_float(~static_cast<uint32_t>(kw[lane * seg + e] >> 32));
-    float incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
+    for (int e = 0; e < kMaxE; ++e) {
+      const int j = lane + 32 * e;
+      pv[e] = (e < E && j < nb) ? exp(srow[j] - mx) : 0.0;
+      esum += pv[e];
     }
-    float run = incl - local;
-    int hit = 0x7fffffff;
-    for (int e = 0; e < seg; ++e) {
-      run += __uint_as_float(~static_cast<uint32_t>(kw[lane * seg + e] >> 32));
-      if (run >= p) {
-        hit = lane * seg + e;
-        break;
+    esum = warp_sum(esum);
+#pragma unroll
+    for (int e = 0; e < kMaxE; ++e) {
+      const int j = lane + 32 * e;
+      pv[e] = (e < E && j < nb) ? pv[e] / esum : -1.0;  // -1: not a key block
+    }
+    // mass(P >= v) and count(P >= v) over this row (the -1 entries never
+    // pass: candidates are non-negative doubles, their bit 62 being clear)
+    auto mass_ge = [&](double v) -> double {
+      double m = 0.0;
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e)
+        if (e < E && pv[e] >= v) m += pv[e];
+      return warp_sum(m);
+    };
+    auto count_ge = [&](double v) -> int {
+      int n = 0;
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e)
+        if (e < E && pv[e] >= v) ++n;
+      return warp_sum_int(n);
+    };
+    auto as_double = [](unsigned long long b) { return __longlong_as_double(static_cast<long long>(b)); };
+    // Top-p: n_p = the length of the shortest prefix, in descending order
+    // (ties: lower index first), whose cumulative mass reaches p; all blocks
+    // when p >= 1 or when the sum never reaches p.
+    int n_p = nb;
+    unsigned long long vsel = 0ull;  // the value at the cut
+    int take = 0;                    // ties of vsel taken, lowest index first
+    bool have_cut = false;
+    if (p < 1.0 && mass_ge(0.0) >= p) {
+      // probabilities lie in [0, 1]: bits 63 (sign) and 62 of their bit
+      // patterns are zero, and the patterns order like the values
+      unsigned long long T = 0ull;
+      for (int b = 61; b >= 0; --b) {
+        const unsigned long long cand = T | (1ull << b);
+        if (mass_ge(as_double(cand)) >= p) T = cand;
+      }
+      // elements above the cut, then ties of the cut value one at a time
+      double m_gt = 0.0;
+      int c_gt = 0, c_eq = 0;
+      const double vT = as_double(T);
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e) {
+        if (e < E) {
+          if (pv[e] > vT) {
+            m_gt += pv[e];
+            ++c_gt;
+          } else if (pv[e] == vT) {
+            ++c_eq;
+          }
+        }
+      }
+      m_gt = warp_sum(m_gt);
+      c_gt = warp_sum_int(c_gt);
+      c_eq = warp_sum_int(c_eq);
+      int m = 0;
+      double acc = m_gt;
+      while (m < c_eq) {
+        acc += vT;
+        ++m;
+        if (acc >= p) break;
+      }
+      n_p = c_gt + m;
+      vsel = T;
+      take = m;
+      have_cut = true;
+    }
+    const int n = min(nb, max(top_k, n_p));
+    if (n == nb) {
+      vsel = 0ull;
+      take = nb;
+      have_cut = false;  // keep everything
+    } else if (n > n_p || !have_cut) {
+      // Top-k floor: the n-th largest by value (ties: lower index first)
+      unsigned long long T = 0ull;
+      for (int b = 61; b >= 0; --b) {
+        const unsigned long long cand = T | (1ull << b);
+        if (count_ge(as_double(cand)) >= n) T = cand;
+      }
+      const double vT = as_double(T);
+      int c_gt = 0;
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e)
+        if (e < E && pv[e] > vT) ++c_gt;
+      c_gt = warp_sum_int(c_gt);
+      vsel = T;
+      take = n - c_gt;
+      have_cut = true;
+    }
+    // mark the selection: everything above vsel, and the first `take` ties
+    // of vsel in index order (j = lane + 32 e: e-major, then lane)
+    const int64_t row = static_cast<int64_t>(bh) * nb + i;
+    const int nwords = E;
+    const double vs = as_double(vsel);
+    int before = 0;  // ties of vsel at lower indices
+    uint32_t myword = 0u;
+#pragma unroll
+    for (int e = 0; e < kMaxE; ++e) {
+      if (e < E) {
+        const bool real = pv[e] >= 0.0;
+        bool keep;
+        if (!have_cut) {
+          keep = real;
+        } else {
+          const bool tie = pv[e] == vs;
+          const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+          const int rank = before + __popc(tb & ((1u << lane) - 1u));
+          keep = pv[e] > vs || (tie && rank < take);
+          before += __popc(tb);
+        }
+        const uint32_t w = __ballot_sync(0xffffffffu, keep);
+        if (lane == e) myword = w;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) hit = min(hit, __shfl_xor_sync(0xffffffffu, hit, o));
-    int n_p = (p >= 1.0f || hit >= nb) ? nb : hit + 1;
-    const int n = min(nb, max(top_k, n_p));
-    for (int e = lane; e < n; e += 32) {
-      const uint32_t j = static_cast<uint32_t>(kw[e] & 0xffffffffu);
-      atomicOr(&words[j >> 5], 1u << (j & 31));
-    }
-    __syncwarp();
-    const int64_t row = static_cast<int64_t>(bh) * nb + i;
-    const int nwords = (nb + 31) >> 5;
-    if (lane < nwords) bitmask[row * nwords + lane] = words[lane];
+    if (lane < nwords) bitmask[row * nwords + lane] = myword;
     if (lane == 0) row_cnt[row] = n;
     __syncwarp();
   }
@@ -421,12 +484,10 @@ cudaError_t launch_scan_expand(const sba_plan* p, const uint32_t* bitmask, const
   const int nb = p->info.nb;
   const int BH = p->g.B * p->g.H;
   const size_t scan_smem = (static_cast<size_t>(kScanWarps) * (nb + 1) + 2 * static_cast<size_t>(BH)) * sizeof(int);
-  static thread_local int configured_scan = 0;
-  if (scan_smem > 48 * 1024 && configured_scan < static_cast<int>(scan_smem)) {
+  if (scan_smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(scan_smem));
     if (e != cudaSuccess) return e;
-    configured_scan = static_cast<int>(scan_smem);
   }
   scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, nb, BH, row_cnt, row_ptr, work_order,
                                                         status);
@@ -438,23 +499,15 @@ cudaError_t launch_scan_expand(const sba_plan* p, const uint32_t* bitmask, const
 
 }  // namespace
 
-static size_t select_smem_bytes(int d, int nkp) {
-  const int ld = d + 4;
-  size_t b = static_cast<size_t>(kRQ) * ld * 4 + static_cast<size_t>(kRQ) * nkp * 4;
-  b += std::max(static_cast<size_t>(kKC) * ld * 4, static_cast<size_t>(kSelWarps) * nkp * 8);
-  b += kSelWarps * 32 * 4;
-  return b;
+static size_t select_smem_bytes(int d, int nb) {
+  return static_cast<size_t>(kRQ) * d * sizeof(double) + static_cast<size_t>(kRQ) * nb * sizeof(double);
 }
 
 cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
                               const float* top_p, int top_k, uint32_t* bitmask, int32_t* row_cnt,
                               int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
-                              void* workspace, cudaStream_t st) {
+                              double* qbar, double* kbar, uint32_t* status, cudaStream_t st) {
   KGeom g = make_kgeom(p);
-  char* ws = static_cast<char*>(workspace);
-  float* qbar = reinterpret_cast<float*>(ws + p->ws_qbar);
-  float* kbar = reinterpret_cast<float*>(ws + p->ws_kbar);
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(ws + p->ws_ctrl);
   const int BH = g.B * g.H;
 
   dim3 pg(g.nb, BH, 2);
@@ -467,24 +520,20 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  int nkp = 32;
-  while (nkp < g.nb) nkp <<= 1;
-  const size_t sel_smem = select_smem_bytes(g.d, nkp);
-  static thread_local int configured_sel = 0;
-  if (sel_smem > 48 * 1024 && configured_sel < static_cast<int>(sel_smem)) {
+  const size_t sel_smem = select_smem_bytes(g.d, g.nb);
+  if (sel_smem > 48 * 1024) {
     e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sel_smem));
     if (e != cudaSuccess) return e;
-    configured_sel = static_cast<int>(sel_smem);
   }
   SelectArgs sa;
   for (int h = 0; h < 256; ++h) sa.top_p[h] = h < g.H ? top_p[h] : 1.0f;
   dim3 sg((g.nb + kRQ - 1) / kRQ, BH);
-  select_kernel<<<sg, kSelThreads, sel_smem, st>>>(g, qbar, kbar, sa, top_k, nkp, bitmask, row_cnt);
+  select_kernel<<<sg, kSelThreads, sel_smem, st>>>(g, qbar, kbar, sa, top_k, bitmask, row_cnt);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order, &ctrl->status, st);
+  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order, status, st);
 }
 
 // ------------------------------------------------------------ stripe masks
@@ -573,88 +622,48 @@ cudaError_t launch_build_stripe_mask(const sba_plan* p, const sba_stripe* params
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_mask_scratch[kNoAllocScratchBytes];
 
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
 
-// Device address of g_mask_scratch on the current device. The lookup runs once
-// per device, on that device's first call (host code must never pass the
-// symbol itself to a kernel: on the host it only names a stand-in).
-cudaError_t scratch_address(void** out) {
+// Device address of g_mask_scratch on the current device (host code must
+// never pass the symbol itself to a kernel: on the host it only names a
+// stand-in). Outside stream capture the address is looked up on every call
+// (cheap, and right again after a device reset reloads the module); a failed
+// lookup is returned and not remembered. Inside a capture, where the lookup
+// may not be allowed, the last successful lookup on this device is used.
+cudaError_t scratch_address(cudaStream_t st, void** out) {
+  *out = nullptr;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_scratch_once[dev], [dev] {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs == cudaStreamCaptureStatusNone) {
     void* ptr = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&ptr, g_mask_scratch);
-    g_scratch_addr[dev] = g_scratch_err[dev] == cudaSuccess ? ptr : nullptr;
-  });
+    e = cudaGetSymbolAddress(&ptr, g_mask_scratch);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    g_scratch_addr[dev] = ptr;
+    *out = ptr;
+    return cudaSuccess;
+  }
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
   *out = g_scratch_addr[dev];
-  return g_scratch_err[dev];
+  return *out ? cudaSuccess : cudaErrorStreamCaptureUnsupported;
 }
 
-size_t noalloc_scratch_need(const sba_plan* p) {
-  const size_t pooled = (static_cast<size_t>(p->info.rows) * p->g.d * sizeof(float) + 255) & ~size_t(255);
-  return sizeof(Ctrl) + 2 * pooled;
+size_t noalloc_pooled_bytes(const sba_plan* p) {
+  return (static_cast<size_t>(p->info.rows) * p->g.d * sizeof(double) + 255) & ~size_t(255);
 }
 
-// The same four launches as launch_build_mask, with the scratch pointers given.
-cudaError_t launch_build_mask_scratch(const sba_plan* p, const void* qt, const void* kt,
-                                      const float* top_p, int top_k, uint32_t* bitmask,
-                                      int32_t* row_cnt, int32_t* row_ptr, int32_t* col_idx,
-                                      int32_t* work_order, char* scratch, cudaStream_t st) {
-  KGeom g = make_kgeom(p);
-  const size_t pooled = (static_cast<size_t>(p->info.rows) * p->g.d * sizeof(float) + 255) & ~size_t(255);
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(scratch);
-  float* qbar = reinterpret_cast<float*>(scratch + sizeof(Ctrl));
-  float* kbar = reinterpret_cast<float*>(scratch + sizeof(Ctrl) + pooled);
-  const int BH = g.B * g.H;
-  // the control block keeps the previous call's contents: start from zero
-  cudaError_t e = cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), st);
-  if (e != cudaSuccess) return e;
-  dim3 pg(g.nb, BH, 2);
-  if (p->g.dtype == SBA_BF16)
-    pool_kernel<__nv_bfloat16><<<pg, kPoolThreads, 0, st>>>(g, static_cast<const char*>(qt),
-                                                            static_cast<const char*>(kt), qbar, kbar);
-  else
-    pool_kernel<float><<<pg, kPoolThreads, 0, st>>>(g, static_cast<const char*>(qt),
-                                                    static_cast<const char*>(kt), qbar, kbar);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  int nkp = 32;
-  while (nkp < g.nb) nkp <<= 1;
-  const size_t sel_smem = select_smem_bytes(g.d, nkp);
-  if (sel_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sel_smem));
-    if (e != cudaSuccess) return e;
-  }
-  SelectArgs sa;
-  for (int h = 0; h < 256; ++h) sa.top_p[h] = h < g.H ? top_p[h] : 1.0f;
-  dim3 sg((g.nb + kRQ - 1) / kRQ, BH);
-  select_kernel<<<sg, kSelThreads, sel_smem, st>>>(g, qbar, kbar, sa, top_k, nkp, bitmask, row_cnt);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int R = p->info.rows;
-  const size_t scan_smem = (static_cast<size_t>(kScanWarps) * (g.nb + 1) + 2 * static_cast<size_t>(BH)) * sizeof(int);
-  if (scan_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(scan_smem));
-    if (e != cudaSuccess) return e;
-  }
-  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, g.nb, BH, row_cnt, row_ptr, work_order,
-                                                        &ctrl->status);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  expand_kernel<<<(R + 7) / 8, 256, 0, st>>>(R, g.nb, bitmask, row_ptr, col_idx);
-  return cudaGetLastError();
-}
+size_t noalloc_scratch_need(const sba_plan* p) { return sizeof(Ctrl) + 2 * noalloc_pooled_bytes(p); }
 
 }  // namespace
 
@@ -665,6 +674,7 @@ extern "C" sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* q
                                              int32_t* row_cnt, int32_t* row_ptr, int32_t* col_idx,
                                              int32_t* work_order, void* stream) {
   using namespace sba;
+  set_error("");
   if (!plan || !qt || !kt || !top_p || !bitmask || !row_cnt || !row_ptr || !col_idx || !work_order) {
     set_error("sba_build_mask_noalloc: NULL argument");
     return SBA_ERR_INVALID_ARG;
@@ -686,23 +696,63 @@ extern "C" sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* q
   }
   const size_t need = noalloc_scratch_need(plan);
   if (need > kNoAllocScratchBytes) {
-    set_error("sba_build_mask_noalloc needs %zu bytes of scratch (2*B*H*nb*d floats + 256) but "
+    set_error("sba_build_mask_noalloc needs %zu bytes of scratch (2*B*H*nb*d doubles + 256) but "
               "its static scratch holds %zu; use sba_build_mask with a workspace",
               need, kNoAllocScratchBytes);
     return SBA_ERR_CAPACITY;
   }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* scratch = nullptr;
-  cudaError_t e = scratch_address(&scratch);
+  cudaError_t e = scratch_address(st, &scratch);
   if (e != cudaSuccess || !scratch) {
     set_error("cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
     return SBA_ERR_CUDA;
   }
-  e = launch_build_mask_scratch(plan, qt, kt, top_p, top_k, bitmask, row_cnt, row_ptr, col_idx,
-                                work_order, static_cast<char*>(scratch),
-                                static_cast<cudaStream_t>(stream));
+  char* sc = static_cast<char*>(scratch);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(sc);
+  double* qbar = reinterpret_cast<double*>(sc + sizeof(Ctrl));
+  double* kbar = reinterpret_cast<double*>(sc + sizeof(Ctrl) + noalloc_pooled_bytes(plan));
+  // the control block keeps the previous call's contents: start from zero
+  e = cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), st);
+  if (e == cudaSuccess)
+    e = launch_build_mask(plan, qt, kt, top_p, top_k, bitmask, row_cnt, row_ptr, col_idx, work_order,
+                          qbar, kbar, &ctrl->status, st);
   if (e != cudaSuccess) {
     set_error("sba_build_mask_noalloc launch: %s", cudaGetErrorString(e));
     return SBA_ERR_CUDA;
+  }
+  return SBA_OK;
+}
+
+extern "C" sba_status sba_noalloc_status(void* stream) {
+  using namespace sba;
+  set_error("");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  cudaError_t e = scratch_address(st, &scratch);
+  if (e != cudaSuccess || !scratch) {
+    set_error("cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    return SBA_ERR_CUDA;
+  }
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    set_error("cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    return SBA_ERR_CUDA;
+  }
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(scratch, 0, sizeof(word));
+  if (e != cudaSuccess) {
+    set_error("reading the scratch status word: %s", cudaGetErrorString(e));
+    return SBA_ERR_CUDA;
+  }
+  if (word & kStatusTimeout) {
+    set_error("a bounded device wait gave up");
+    return SBA_ERR_DEVICE_TIMEOUT;
+  }
+  if (word & kStatusCheck) {
+    set_error("a device-side input check failed");
+    return SBA_ERR_DEVICE_CHECK;
   }
   return SBA_OK;
 }

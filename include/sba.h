@@ -158,8 +158,8 @@ SBA_API sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o,
 
 /* Block scoring and routing (FVAttn abstract: Top-p routing, Top-k safety
  * floor). For every row r = (b, h, i):
- *   Qbar_i, Kbar_j = means of qt, kt over the real tokens of block i, j (fp32)
- *   P_ij = softmax_j(Qbar_i . Kbar_j / sqrt(d))
+ *   Qbar_i, Kbar_j = means of qt, kt over the real tokens of block i, j (fp64)
+ *   P_ij = softmax_j(Qbar_i . Kbar_j / sqrt(d))   (fp64)
  *   sort j by P_ij descending (ties: lower j first); n_p = the shortest
  *   prefix whose cumulative mass reaches top_p[h] (all nb when it never does
  *   or top_p[h] >= 1); keep n = min(nb, max(top_k, n_p)) blocks.
@@ -175,8 +175,12 @@ SBA_API sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o,
  *             (ties: lower row first). Rows that run together then share one
  *             head's keys and values in L2.
  * top_p is a host array [H]; values in (0, 1] are meaningful, p >= 1 keeps
- * every block. top_k >= 0. Scores are fp32; rows whose cumulative mass at the
- * cut lies within ~1e-5 of p may differ from an fp64 evaluation. */
+ * every block. top_k >= 0. Pooling, scores, softmax and the cumulative mass
+ * are fp64 (the cut is found by bisection on the probabilities, not by a
+ * sort), so a row can differ from another fp64 evaluation only where its
+ * cumulative mass at the cut lies within rounding (~1e-15) of p.
+ * The workspace holds the pooled means (2*B*H*nb*d doubles) and the status
+ * word that device-side checks set. */
 SBA_API sba_status sba_build_mask(const sba_plan* plan, const void* qt, const void* kt,
                           const float* top_p, int32_t top_k,
                           uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
@@ -186,25 +190,34 @@ SBA_API sba_status sba_build_mask(const sba_plan* plan, const void* qt, const vo
 /* Allocation-free sba_build_mask (the paper has no counterpart: this is a
  * deployment convenience). Same inputs, outputs and results as sba_build_mask,
  * but no workspace argument: its scratch (the pooled block means and a
- * 256-byte control block) lives in one 32 MiB array of static device memory
+ * 256-byte control block) lives in one 64 MiB array of static device memory
  * inside the library, which every GPU that loads libsba holds until the
  * process exits. For callers that cannot allocate device memory or carry a
  * workspace: plugin interfaces that pass only inputs and outputs, and services
  * that reserve all device memory at start-up and forbid cudaMalloc afterwards.
- * Limit: 2*B*H*nb*d*4 bytes (rounded up to 256 each) + 256 <= 32 MiB, i.e.
+ * Limit: 2*B*H*nb*d*8 bytes (rounded up to 256 each) + 256 <= 64 MiB, i.e.
  * B*H*nb*d <= ~4.19 million (the Wan and HunyuanVideo-shaped layers fit);
  * larger plans return SBA_ERR_CAPACITY before anything is launched.
- * The first call on each device looks up the array's device address with
- * cudaGetSymbolAddress (make that first call before any stream capture).
- * Each call clears the control block with cudaMemsetAsync and overwrites the
- * pooled means; the array keeps the last call's contents. All calls share the
- * one array, so calls that overlap on the GPU (other streams, other threads)
- * race: serialise them. Never calls cudaMalloc, cudaFree or any allocating
+ * Each call looks up the array's device address on the current device with
+ * cudaGetSymbolAddress (a failed lookup is reported, not remembered); inside a
+ * stream capture it reuses the last address found on that device, so make one
+ * call on each device before capturing. Each call clears the control block
+ * with cudaMemsetAsync and overwrites the pooled means; the array keeps the
+ * last call's contents. All calls share the one array, so calls that overlap
+ * on the GPU (other streams, other threads) race: serialise them. Device-side
+ * check failures of the call land in the array's status word: read them with
+ * sba_noalloc_status. Never calls cudaMalloc, cudaFree or any allocating
  * routine. */
 SBA_API sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* qt, const void* kt,
                                           const float* top_p, int32_t top_k,
                                           uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
                                           int32_t* col_idx, int32_t* work_order, void* stream);
+
+/* Status word of sba_build_mask_noalloc's static scratch (no counterpart in
+ * the paper): synchronise `stream`, read and clear the word. Returns SBA_OK,
+ * SBA_ERR_DEVICE_TIMEOUT or SBA_ERR_DEVICE_CHECK like
+ * sba_check_device_status, or SBA_ERR_CUDA. */
+SBA_API sba_status sba_noalloc_status(void* stream);
 
 /* Stripe mask (Parameterized Stripe Attention for Efficient Video Generation,
  * Approach: a six-parameter mask M(Tw, To, Ts, Sw, So, Ss) of periodic

@@ -265,21 +265,20 @@ def select_row(P: np.ndarray, p: float, k: int):
         "n": n,
         "c_at": float(c[n_p - 1]),
         "c_before": float(c[n_p - 2]) if n_p >= 2 else 0.0,
-        "gap": float(P[order[n - 1]] - P[order[n]]) if n < nkb else math.inf,
         "order": order,
     }
     return sel, info
 
 
 def build_mask(Qt: np.ndarray, Kt: np.ndarray, g: Geom, top_p, top_k: int,
-               boundary_tol: float = 1e-4, tie_tol: float = 1e-6) -> dict:
+               boundary_tol: float = 1e-4) -> dict:
     """Pool, score, select every (b, h, query block) row; emit bitmask and CSR.
 
     Rows are flattened as r = (b*H + h)*nb + i. ``col_idx`` is ascending inside
     each row. Bit j of a row lives in word j//32 at position j%32.
     ``boundary`` marks rows whose cumulative mass at the cut lies within
-    ``boundary_tol`` of p; ``near_tie`` rows whose last kept and first dropped
-    probabilities differ by at most ``tie_tol``.
+    ``boundary_tol`` of p (the only rows where another correct fp64
+    evaluation may cut elsewhere).
     """
     B, H = Qt.shape[:2]
     nb = g.nb
@@ -289,7 +288,6 @@ def build_mask(Qt: np.ndarray, Kt: np.ndarray, g: Geom, top_p, top_k: int,
     row_cnt = np.zeros(R, dtype=np.int64)
     bitmask = np.zeros((R, words), dtype=np.uint32)
     boundary = np.zeros(R, dtype=bool)
-    near_tie = np.zeros(R, dtype=bool)
     cols = []
     for b in range(B):
         for h in range(H):
@@ -304,12 +302,11 @@ def build_mask(Qt: np.ndarray, Kt: np.ndarray, g: Geom, top_p, top_k: int,
                 bitmask[r] = np.packbits(bits, bitorder="little").view("<u4")
                 boundary[r] = (abs(info["c_at"] - p) <= boundary_tol
                                or abs(info["c_before"] - p) <= boundary_tol)
-                near_tie[r] = info["gap"] <= tie_tol
     row_ptr = np.zeros(R + 1, dtype=np.int64)
     row_ptr[1:] = np.cumsum(row_cnt)
     col_idx = np.concatenate(cols).astype(np.int64) if cols else np.zeros(0, np.int64)
     return {"probs": Pm, "row_cnt": row_cnt, "row_ptr": row_ptr, "col_idx": col_idx,
-            "bitmask": bitmask, "boundary": boundary, "near_tie": near_tie}
+            "bitmask": bitmask, "boundary": boundary}
 
 
 def lpt_order(row_cnt: np.ndarray, nb: int) -> np.ndarray:

@@ -52,6 +52,10 @@ def test_noalloc_mask_equals_workspace_mask_on_two_calls_in_a_row():
     for r, g in zip(ref, got):
         for key in r:
             assert np.array_equal(r[key], g[key]), key
+    # the device-side checks of those calls found nothing, and reading the
+    # status clears it
+    assert sba.sba_noalloc_status() == sba.SBA_OK
+    assert sba.sba_noalloc_status() == sba.SBA_OK
 
 
 def test_noalloc_rejects_a_plan_larger_than_its_scratch():
