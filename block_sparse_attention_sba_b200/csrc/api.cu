@@ -54,6 +54,12 @@ KGeom make_kgeom(const sba_plan* p) {
   k.dv_nH = DivMod(k.nH);
   k.dv_H = DivMod(G.H);
   k.dv_nb = DivMod(k.nb);
+  const int vh_e = G.Hh - (k.nH - 1) * G.ch, vw_e = G.W - (k.nW - 1) * G.cw;
+  for (int he = 0; he < 2; ++he)
+    for (int we = 0; we < 2; ++we)
+      k.dv_area[he * 2 + we] = DivMod((he ? vh_e : G.ch) * (we ? vw_e : G.cw));
+  k.dv_w[0] = DivMod(G.cw);
+  k.dv_w[1] = DivMod(vw_e);
   return k;
 }
 

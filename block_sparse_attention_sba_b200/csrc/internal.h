@@ -61,6 +61,9 @@ struct KGeom {
   int32_t tail;   // Hilbert order: real tokens in the last block
   int64_t sB, sH, sN;
   DivMod dv_cw, dv_chcw, dv_nW, dv_nH, dv_H, dv_nb;
+  // in-cube rank divisors of the cube kinds along h and w: index
+  // (last cube along h) * 2 + (last cube along w); area = vh*vw, then vw
+  DivMod dv_area[4], dv_w[2];
 };
 
 KGeom make_kgeom(const sba_plan* p);

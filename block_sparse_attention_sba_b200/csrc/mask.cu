@@ -127,7 +127,7 @@ __device__ __forceinline__ int warp_sum_int(int v) {
 // bisection on the bit pattern of v (warp mass sums), the ties of v taken in
 // index order until the mass reaches p; the Top-k floor by the same
 // bisection on counts. No sort.
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 2)
     select_kernel(KGeom g, const double* __restrict__ qbar, const double* __restrict__ kbar,
                   SelectArgs sa, int top_k, uint32_t* __restrict__ bitmask,
                   int32_t* __restrict__ row_cnt) {
@@ -197,23 +197,63 @@ __global__ void __launch_bounds__(kSelThreads)
       const int j = lane + 32 * e;
       pv[e] = (e < E && j < nb) ? pv[e] / esum : -1.0;  // -1: not a key block
     }
-    // mass(P >= v) and count(P >= v) over this row (the -1 entries never
-    // pass: candidates are non-negative doubles, their bit 62 being clear)
-    auto mass_ge = [&](double v) -> double {
-      double m = 0.0;
+    // mass and count of the row's probabilities >= v (the -1 entries never
+    // pass: every v tried is a non-negative double, bit 62 of its pattern
+    // being clear)
+    auto ge_sums = [&](double v, double& m, int& c) {
+      double mm = 0.0;
+      int cc = 0;
 #pragma unroll
       for (int e = 0; e < kMaxE; ++e)
-        if (e < E && pv[e] >= v) m += pv[e];
-      return warp_sum(m);
-    };
-    auto count_ge = [&](double v) -> int {
-      int n = 0;
+        if (e < E && pv[e] >= v) {
+          mm += pv[e];
+          ++cc;
+        }
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e)
-        if (e < E && pv[e] >= v) ++n;
-      return warp_sum_int(n);
+      for (int o = 16; o > 0; o >>= 1) {
+        mm += __shfl_xor_sync(0xffffffffu, mm, o);
+        cc += __shfl_xor_sync(0xffffffffu, cc, o);
+      }
+      m = mm;
+      c = cc;
     };
     auto as_double = [](unsigned long long b) { return __longlong_as_double(static_cast<long long>(b)); };
+    // The single probability in [lo, hi) (bit patterns), found once the
+    // bisection interval holds exactly one element.
+    auto only_in = [&](unsigned long long lo, unsigned long long hi) -> unsigned long long {
+      double f = -1.0;
+      const double a = as_double(lo), b = as_double(hi);
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e)
+        if (e < E && pv[e] >= a && pv[e] < b) f = pv[e];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) f = fmax(f, __shfl_xor_sync(0xffffffffu, f, o));
+      return static_cast<unsigned long long>(__double_as_longlong(f));
+    };
+    // Bisection over bit patterns for the largest element v with
+    // pred(mass(P >= v), count(P >= v)). Invariant: pred holds at lo and fails
+    // at hi, so the answer lies in [lo, hi); stop once one element is left
+    // there (or the interval is one pattern wide).
+    auto bisect = [&](bool by_mass, double p_or_n) -> unsigned long long {
+      unsigned long long lo = 0ull, hi = 1ull << 62;
+      double m;
+      int c_lo, c_hi = 0;
+      ge_sums(0.0, m, c_lo);
+      for (int b = 61; b >= 0 && c_lo - c_hi > 1; --b) {
+        const unsigned long long mid = lo | (1ull << b);
+        int c;
+        ge_sums(as_double(mid), m, c);
+        const bool ok = by_mass ? (m >= p_or_n) : (static_cast<double>(c) >= p_or_n);
+        if (ok) {
+          lo = mid;
+          c_lo = c;
+        } else {
+          hi = mid;
+          c_hi = c;
+        }
+      }
+      return c_lo - c_hi == 1 ? only_in(lo, hi) : lo;
+    };
     // Top-p: n_p = the length of the shortest prefix, in descending order
     // (ties: lower index first), whose cumulative mass reaches p; all blocks
     // when p >= 1 or when the sum never reaches p.
@@ -221,14 +261,11 @@ __global__ void __launch_bounds__(kSelThreads)
     unsigned long long vsel = 0ull;  // the value at the cut
     int take = 0;                    // ties of vsel taken, lowest index first
     bool have_cut = false;
-    if (p < 1.0 && mass_ge(0.0) >= p) {
-      // probabilities lie in [0, 1]: bits 63 (sign) and 62 of their bit
-      // patterns are zero, and the patterns order like the values
-      unsigned long long T = 0ull;
-      for (int b = 61; b >= 0; --b) {
-        const unsigned long long cand = T | (1ull << b);
-        if (mass_ge(as_double(cand)) >= p) T = cand;
-      }
+    double total;
+    int cnt_all;
+    ge_sums(0.0, total, cnt_all);
+    if (p < 1.0 && total >= p) {
+      const unsigned long long T = bisect(true, p);
       // elements above the cut, then ties of the cut value one at a time
       double m_gt = 0.0;
       int c_gt = 0, c_eq = 0;
@@ -266,11 +303,7 @@ __global__ void __launch_bounds__(kSelThreads)
       have_cut = false;  // keep everything
     } else if (n > n_p || !have_cut) {
       // Top-k floor: the n-th largest by value (ties: lower index first)
-      unsigned long long T = 0ull;
-      for (int b = 61; b >= 0; --b) {
-        const unsigned long long cand = T | (1ull << b);
-        if (count_ge(as_double(cand)) >= n) T = cand;
-      }
+      const unsigned long long T = bisect(false, static_cast<double>(n));
       const double vT = as_double(T);
       int c_gt = 0;
 #pragma unroll

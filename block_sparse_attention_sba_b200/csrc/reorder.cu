@@ -46,7 +46,10 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(KGeom g, ReorderArgs 
   // real sub-box of this cube; its tokens fill slots [0, len) row-major
   const int vh = min(g.ch, g.Hh - h0), vw = min(g.cw, g.W - w0);
   const int len = min(g.ct, g.T - t0) * vh * vw;
-  const bool full = len == g.bs;
+  // in-cube offsets are ranks over the real sub-box: (vh*vw, vw) divisors
+  const int he = static_cast<int>(th) == g.nH - 1, we = static_cast<int>(tw) == g.nW - 1;
+  const DivMod dv_area = g.dv_area[he * 2 + we];
+  const DivMod dv_w = g.dv_w[we];
 
   const int64_t row_bytes = static_cast<int64_t>(g.d) * esize;
   const int64_t packed_base = (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * row_bytes;
@@ -73,25 +76,12 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(KGeom g, ReorderArgs 
       valid = tok >= 0;
       n = tok;
     } else {
-      int lt, lh, lw;
-      if (full) {
-        uint32_t a, r2, b, c;
-        g.dv_chcw.divmod(static_cast<uint32_t>(o), a, r2);
-        g.dv_cw.divmod(r2, b, c);
-        lt = static_cast<int>(a);
-        lh = static_cast<int>(b);
-        lw = static_cast<int>(c);
-      } else {
-        // edge cube: rank o among the real sub-box's tokens (plain division;
-        // only the edge cubes of the grid take this branch)
-        const int area = vh * vw;
-        lt = o / area;
-        const int r2 = o - lt * area;
-        lh = r2 / vw;
-        lw = r2 - lh * vw;
-      }
+      uint32_t lt, r2, lh, lw;
+      dv_area.divmod(static_cast<uint32_t>(o), lt, r2);
+      dv_w.divmod(r2, lh, lw);
       valid = o < len;
-      n = (static_cast<int64_t>(t0 + lt) * g.Hh + (h0 + lh)) * g.W + (w0 + lw);
+      n = (static_cast<int64_t>(t0 + static_cast<int>(lt)) * g.Hh + (h0 + static_cast<int>(lh))) * g.W +
+          (w0 + static_cast<int>(lw));
     }
     const int64_t raster = raster_base + n * sN_bytes + c * 16;
     const int64_t packed = packed_base + static_cast<int64_t>(o) * row_bytes + c * 16;
