@@ -269,11 +269,34 @@ def run_reference(args):
     return 0
 
 
+def sm_idle_fraction(tr, nsm: int) -> float:
+    """SM idle / tail fraction from per-row (start, end, smid) stamps:
+    1 - sum over SMs of the time the SM had at least one row in flight /
+    (SMs x makespan). Rows that overlap on one SM (the attention kernel runs
+    two at once per CTA) count once."""
+    import numpy as np
+    tr = np.asarray(tr, dtype=np.int64).reshape(-1, 3)
+    t0, t1 = int(tr[:, 0].min()), int(tr[:, 1].max())
+    busy = 0
+    for sm in np.unique(tr[:, 2]):
+        iv = tr[tr[:, 2] == sm][:, :2]
+        iv = iv[np.argsort(iv[:, 0], kind="stable")]
+        cur_s, cur_e = int(iv[0, 0]), int(iv[0, 1])
+        for s, e in iv[1:]:
+            if s > cur_e:
+                busy += cur_e - cur_s
+                cur_s, cur_e = int(s), int(e)
+            else:
+                cur_e = max(cur_e, int(e))
+        busy += cur_e - cur_s
+    return 1.0 - busy / (nsm * float(t1 - t0))
+
+
 def sched_report(dev, name="stress", reps=3):
     """SM idle / tail fraction of sba_attention on the heterogeneous-load
-    workload, persistent longest-first vs one CTA per row in head-major order,
-    from per-row %globaltimer stamps: idle = 1 - sum(row busy time) /
-    (SMs x makespan). Also the per-head spread of selected blocks."""
+    workload, persistent longest-first vs a grid in head-major order (two rows
+    per CTA), from per-row %globaltimer stamps (see sm_idle_fraction). Also
+    the per-head spread of selected blocks."""
     import torch
 
     import block_sparse_attention_sba_b200 as sba
@@ -300,11 +323,8 @@ def sched_report(dev, name="stress", reps=3):
             e1.record()
             torch.cuda.synchronize(dev)
             tr = trace.view(R, 3).cpu()
-            t0 = int(tr[:, 0].min())
-            t1 = int(tr[:, 1].max())
-            busy = float((tr[:, 1] - tr[:, 0]).sum())
-            span = float(t1 - t0)
-            res = {"ms": e0.elapsed_time(e1), "idle_frac": 1.0 - busy / (nsm * span),
+            span = float(int(tr[:, 1].max()) - int(tr[:, 0].min()))
+            res = {"ms": e0.elapsed_time(e1), "idle_frac": sm_idle_fraction(tr.numpy(), nsm),
                    "makespan_ms": span * 1e-6, "sms_used": int(torch.unique(tr[:, 2]).numel())}
             if best is None or res["ms"] < best["ms"]:
                 best = res
@@ -584,8 +604,7 @@ def report_all(args):
                               sa.lse, mode, trace, sa.workspace)
             torch.cuda.synchronize(dev)
             tr = trace.view(R, 3).cpu()
-            span = float(tr[:, 1].max() - tr[:, 0].min())
-            idle[label] = 1.0 - float((tr[:, 1] - tr[:, 0]).sum()) / (nsm * span)
+            idle[label] = sm_idle_fraction(tr.numpy(), nsm)
         rb, mb, ub = _alg_bytes(wl, plan.info)
         att_s = ms["attention"] * 1e-3
         line = {"workload": name, "dtype": wl.dtype, "ms": {k2: round(v2, 4) for k2, v2 in ms.items()},

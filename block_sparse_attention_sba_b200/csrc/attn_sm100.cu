@@ -125,6 +125,7 @@ struct AttnParams {
   Ctrl* ctrl;
   int R;
   int sched;
+  int64_t max_nnz;  // col_idx capacity the plan guarantees (B*H*nb*nb)
   uint64_t budget_ns;
   float scale_log2;
   // low-bit path only
@@ -242,9 +243,11 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       if (row >= 0) {
         start = __ldg(&P.row_ptr[row]);
         n = __ldg(&P.row_ptr[row + 1]) - start;
-        if (n < 0 || n > g.nb) {
+        if (n < 0 || n > g.nb || start < 0 || static_cast<int64_t>(start) + n > P.max_nnz) {
+          // a row that cannot be read is skipped (written as empty)
           if (lane == 0) atomicOr(status, kStatusCheck);
-          n = n < 0 ? 0 : g.nb;
+          n = 0;
+          start = 0;
         }
       }
       const int rs = items & 1;
@@ -777,11 +780,13 @@ __global__ void __launch_bounds__(128)
     o[c] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int start = row_ptr[row];
+  int start = row_ptr[row];
   int n = row_ptr[row + 1] - start;
-  if (n < 0 || n > g.nb) {
+  if (n < 0 || n > g.nb || start < 0 || static_cast<int64_t>(start) + n > static_cast<int64_t>(g.nb) * g.nb * g.B * g.H) {
+    // a row that cannot be read is skipped (written as empty)
     if (t == 0) atomicOr(status, kStatusCheck);
-    n = n < 0 ? 0 : g.nb;
+    n = 0;
+    start = 0;
   }
   for (int i = 0; i < n; ++i) {
     int j = col_idx[start + i];
@@ -923,6 +928,10 @@ cudaError_t launch_tc(const sba_plan* p, const void* qt, const void* kt, const v
 }  // namespace
 
 int attention_grid_size() { return g_grid_size; }
+void note_attention_grid_size(int grid) { g_grid_size = grid; }
+bool tma_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows) {
+  return make_map(map, base, rows, D, box_rows);
+}
 
 cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, const void* vt,
                              const int32_t* row_ptr, const int32_t* col_idx,
@@ -952,10 +961,14 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
   ap.ctrl = ctrl;
   ap.R = p->info.rows;
   ap.sched = sched;
+  ap.max_nnz = p->info.max_nnz;
   ap.budget_ns = p->wait_budget_ns;
   ap.scale_log2 = scale_log2;
   ap.vmean = nullptr;
   ap.vexp = nullptr;
+  if (g.bs == 128)  // two query tiles in flight per CTA
+    return launch_attention_dual(p, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse, sched, trace,
+                                 workspace, st);
   if (g.d == 128 && g.bs == 128) return launch_tc<128, 128>(p, qt, kt, vt, ap, st);
   if (g.d == 128 && g.bs == 64) return launch_tc<128, 64>(p, qt, kt, vt, ap, st);
   if (g.d == 64 && g.bs == 128) return launch_tc<64, 128>(p, qt, kt, vt, ap, st);
@@ -979,6 +992,7 @@ cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const voi
   ap.ctrl = reinterpret_cast<Ctrl*>(static_cast<char*>(workspace) + p->ws_ctrl);
   ap.R = p->info.rows;
   ap.sched = SBA_SCHED_LPT;
+  ap.max_nnz = p->info.max_nnz;
   ap.budget_ns = p->wait_budget_ns;
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(g.d)));
   ap.vmean = vmean;

@@ -33,6 +33,10 @@ SMALL = {
     "hilbert_small": datagen.with_order(datagen.WORKLOADS["small"], "hilbert"),
     "hilbert_f32": datagen.custom("hilbert_f32", 1, 2, 5, 6, 7, 64, (4, 4, 4), dtype="f32",
                                   top_p=(0.9,), top_k=1, order="hilbert"),
+    # 1080 rows (40 heads x 27 blocks, ragged in h and w): several rows per
+    # persistent CTA, so both query tiles of a CTA go through row changes
+    "many_rows_d128": datagen.custom("many_rows_d128", 1, 40, 6, 22, 21, 128, (2, 8, 8),
+                                     top_p=(0.5, 0.9, 0.97), top_k=2, rope_split=(44, 42, 42)),
 }
 
 
@@ -154,25 +158,31 @@ def test_topk_floor_and_cap():
     assert np.all(gpu2["row_cnt"] == g.nb)
 
 
-def _attn_with_csr(wl, q, k, v, row_ptr, col_idx, sched=1):
+def _attn_with_csr(wl, q, k, v, row_ptr, col_idx, sched=1, work_counts=None):
+    """sba_attention on a hand-made CSR; col_idx is held in a buffer of the
+    plan's max_nnz capacity (zero beyond the given entries)."""
     import block_sparse_attention_sba_b200 as sba
     g = geom_of(wl)
     plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube, order=wl.order)
     sa = sba.SparseAttention(plan, device=q.device)
     sba.sba_reorder(plan.handle, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace)
     rp = torch.tensor(row_ptr, dtype=torch.int32, device=q.device)
-    ci = torch.tensor(col_idx if len(col_idx) else [0], dtype=torch.int32, device=q.device)
-    wo = torch.tensor(oracle.lpt_order(np.diff(row_ptr), g.nb), dtype=torch.int32, device=q.device)
+    ci = torch.zeros(plan.info.max_nnz, dtype=torch.int32, device=q.device)
+    if len(col_idx):
+        ci[:len(col_idx)] = torch.tensor(col_idx, dtype=torch.int32, device=q.device)
+    counts = np.diff(row_ptr) if work_counts is None else work_counts
+    wo = torch.tensor(oracle.lpt_order(counts, g.nb), dtype=torch.int32, device=q.device)
     sba.sba_attention(plan.handle, sa.qt, sa.kt, sa.vt, rp, ci, wo, sa.ot, sa.lse, sched, None,
                       sa.workspace)
     torch.cuda.synchronize()
     return sa, sa.check()
 
 
+@pytest.mark.parametrize("name", ["ragged_d128_bs64", "ragged_d128_bs128", "ragged_d64_bs128"])
 @pytest.mark.parametrize("sched", [0, 1])
-def test_handmade_csr_with_empty_and_single_block_rows(sched):
-    wl = SMALL["ragged_d128_bs64"]
-    q, k, v = _inputs("ragged_d128_bs64", wl)
+def test_handmade_csr_with_empty_and_single_block_rows(sched, name):
+    wl = SMALL[name]
+    q, k, v = _inputs(name, wl)
     g = geom_of(wl)
     R = wl.B * wl.H * g.nb
     rng = np.random.default_rng(5)
@@ -207,9 +217,10 @@ def test_handmade_csr_with_empty_and_single_block_rows(sched):
             assert np.all(np.isneginf(lse[b, h, sl][valid[sl]]))
 
 
-def test_out_of_range_column_sets_device_check_and_context_survives():
-    wl = SMALL["small"]
-    q, k, v = _inputs("small", wl)
+@pytest.mark.parametrize("name", ["small", "ragged_d128_bs128"])
+def test_out_of_range_column_sets_device_check_and_context_survives(name):
+    wl = SMALL[name]
+    q, k, v = _inputs(name, wl)
     g = geom_of(wl)
     R = wl.B * wl.H * g.nb
     row_ptr = np.arange(R + 1)
@@ -222,6 +233,41 @@ def test_out_of_range_column_sets_device_check_and_context_survives():
     sa2, status2 = _attn_with_csr(wl, q, k, v, row_ptr, np.zeros(R, dtype=np.int64), sched=0)
     assert status2 == 0
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("name", ["small", "ragged_d128_bs128"])
+@pytest.mark.parametrize("sched", [0, 1])
+def test_corrupt_row_pointers_are_skipped_and_flagged(name, sched):
+    """Row pointers that give a negative length, more than nb columns or a
+    start past the plan's col_idx capacity make their rows empty and set
+    SBA_ERR_DEVICE_CHECK; every other row is still computed, and nothing is
+    read outside the col_idx buffer (it holds max_nnz entries)."""
+    wl = SMALL[name]
+    q, k, v = _inputs(name, wl)
+    g = geom_of(wl)
+    R = wl.B * wl.H * g.nb
+    row_ptr = np.arange(R + 1, dtype=np.int64)
+    col_idx = np.arange(R, dtype=np.int64) % g.nb
+    good_counts = np.ones(R, dtype=np.int64)
+    row_ptr[5] = row_ptr[5] + 3       # row 4: four columns (valid); row 5: length -2
+    row_ptr[R] = 1 << 30              # row R-1: far more than nb columns
+    import block_sparse_attention_sba_b200 as sba
+    sa, status = _attn_with_csr(wl, q, k, v, row_ptr, col_idx, sched=sched, work_counts=good_counts)
+    assert status == sba.SBA_ERR_DEVICE_CHECK
+    ot = sa.ot.cpu()
+    for r in (5, R - 1):
+        b, h, i = r // (wl.H * g.nb), (r // g.nb) % wl.H, r % g.nb
+        assert torch.all(ot[b, h, i * g.bs:(i + 1) * g.bs] == 0)
+    # a good row computed in the same launch matches the oracle
+    qt, kt, vt = (to64(x.cpu()) for x in (sa.qt, sa.kt, sa.vt))
+    rp_ok = np.arange(R + 1)
+    Ot, _ = oracle.attention(qt, kt, vt, g, rp_ok, col_idx, blocks=[(0, 0, 2)])
+    valid = oracle.slot_valid(g)
+    sl = slice(2 * g.bs, 3 * g.bs)
+    mx, rel = attention_errors(to64(ot)[0, 0, sl][valid[sl]], Ot[0, 0, sl][valid[sl]])
+    assert mx <= ATOL and rel <= REL_L2
+    _, status2 = _attn_with_csr(wl, q, k, v, rp_ok, col_idx, sched=sched)
+    assert status2 == 0
 
 
 def test_bounded_wait_gives_up_and_reports_timeout():
