@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 LIB = os.path.join(PKG, "libsba.so")
-SOURCES = ["api.cu", "reorder.cu", "mask.cu", "attn_sm100.cu", "attn_dual.cu", "lowbit.cu"]
+SOURCES = ["api.cu", "reorder.cu", "mask.cu", "attn_sm100.cu", "lowbit.cu"]
 HEADERS = ["internal.h", "ptx.cuh"]
 
 NVCC_FLAGS = [

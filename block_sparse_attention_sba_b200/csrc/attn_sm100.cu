@@ -110,6 +110,7 @@ struct Cfg {
   static_assert(NK >= 2 && NV >= 1, "need K and V slots");
   static_assert(D <= 128 && BS <= 128, "TMEM plan assumes d, bs <= 128");
   static_assert(NBAR * 8 <= 512, "barrier area");
+  static_assert(NK <= 16 && NV <= 16, "slot length records");
   static_assert(1024 + (NSB * NWG + NWG) * 128 * 4 <= CTRL_BYTES, "control area");
   static_assert(SMEM <= kSmemLimit, "shared memory budget");
 };
@@ -161,6 +162,10 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 516);
   int* ring = reinterpret_cast<int*>(ctl + 528);             // [2][4]
+  // real keys of the block each K / V slot holds (written before the slot's
+  // TMA arrive, read after its full barrier)
+  int* klen_k = reinterpret_cast<int*>(ctl + 576);  // [NK]
+  int* klen_v = reinterpret_cast<int*>(ctl + 640);  // [NV]
   float* xmax = reinterpret_cast<float*>(ctl + 1024);        // [NSB][NWG][128] partial row maxima
   float* xsum = xmax + C::NSB * C::NWG * 128;                // [NWG][128] partial row sums
 
@@ -338,6 +343,7 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           }
         }
         if (lane == 0) {
+          (isv ? klen_v : klen_k)[s] = block_len(g, j);
           if (LB && isv) {
             // E4M3 codes of block j, [d][bs] bytes: one 128-byte-wide box
             const uint32_t dst = smem_u32(sV + s * C::VTILE_BYTES);
@@ -403,12 +409,15 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
         if (lane == 0) {
           const uint32_t dS = tmem + static_cast<uint32_t>(b) * 128u;
           const uint32_t k_addr = smem_u32(sK + s * C::TILE_BYTES);
+          // S over the block's real keys only, rounded up to the MMA's N step
+          // of 16 (the softmax masks the rest of the row)
+          const uint32_t idesc_s = idesc_bf16_f32(C::M, (klen_k[s] + 15) & ~15, 0, 0);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk & 3) * 32;
             const uint64_t a = smem_desc_sw128(q_addr + (kk >> 2) * (C::M * 128) + off, 16, 1024);
             const uint64_t bd = smem_desc_sw128(k_addr + (kk >> 2) * (BS * 128) + off, 16, 1024);
-            mma_ss(dS, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+            mma_ss(dS, a, bd, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(C::B_SR + b));
           mma_commit(bar(C::B_KE + s));
@@ -468,10 +477,15 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
                         C::IDESC_MEAN, 1u);
           } else {
             const uint32_t v_addr = smem_u32(sV + s * C::TILE_BYTES);
+            // k-steps of 16 keys up to the block's last real key (P is zero
+            // beyond it)
+            const int nks = (klen_v[s] + 15) >> 4;
 #pragma unroll
             for (int kk = 0; kk < BS / 16; ++kk) {
-              const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, BS * 128, 1024);
-              mma_ts(tmem + C::COL_O, aP + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+              if (kk < nks) {
+                const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, BS * 128, 1024);
+                mma_ts(tmem + C::COL_O, aP + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+              }
             }
           }
           mma_commit(bar(C::B_PD + b));
@@ -537,6 +551,7 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t scol = tmem + lane_off + static_cast<uint32_t>(b) * 128u;
+          const int klen = block_len(g, j);
           uint32_t sr[CPW];
 #pragma unroll
           for (int c = 0; c < CPW / 32; ++c)
@@ -545,7 +560,6 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           float s[CPW];
 #pragma unroll
           for (int e = 0; e < CPW; ++e) s[e] = __uint_as_float(sr[e]);
-          const int klen = block_len(g, j);
           if (klen < BS) {
             // padding keys (slots klen .. BS-1) are masked
 #pragma unroll
@@ -928,10 +942,6 @@ cudaError_t launch_tc(const sba_plan* p, const void* qt, const void* kt, const v
 }  // namespace
 
 int attention_grid_size() { return g_grid_size; }
-void note_attention_grid_size(int grid) { g_grid_size = grid; }
-bool tma_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows) {
-  return make_map(map, base, rows, D, box_rows);
-}
 
 cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, const void* vt,
                              const int32_t* row_ptr, const int32_t* col_idx,
@@ -966,9 +976,6 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
   ap.scale_log2 = scale_log2;
   ap.vmean = nullptr;
   ap.vexp = nullptr;
-  if (g.bs == 128)  // two query tiles in flight per CTA
-    return launch_attention_dual(p, qt, kt, vt, row_ptr, col_idx, work_order, ot, lse, sched, trace,
-                                 workspace, st);
   if (g.d == 128 && g.bs == 128) return launch_tc<128, 128>(p, qt, kt, vt, ap, st);
   if (g.d == 128 && g.bs == 64) return launch_tc<128, 64>(p, qt, kt, vt, ap, st);
   if (g.d == 64 && g.bs == 128) return launch_tc<64, 128>(p, qt, kt, vt, ap, st);

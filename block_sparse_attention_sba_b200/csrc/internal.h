@@ -108,19 +108,8 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
                              const int32_t* row_ptr, const int32_t* col_idx,
                              const int32_t* work_order, void* ot, float* lse, int sched,
                              uint64_t* trace, void* workspace, cudaStream_t st);
-// bf16 block size 128: two query tiles in flight per CTA (attn_dual.cu).
-cudaError_t launch_attention_dual(const sba_plan* p, const void* qt, const void* kt, const void* vt,
-                                  const int32_t* row_ptr, const int32_t* col_idx,
-                                  const int32_t* work_order, void* ot, float* lse, int sched,
-                                  uint64_t* trace, void* workspace, cudaStream_t st);
 cudaError_t launch_timeout_probe(void* workspace, uint64_t timeout_ns, cudaStream_t st);
 
-// 2-D tensor map over a bf16 [rows][D] tensor, boxes of 64 columns x
-// box_rows rows, 128-byte swizzle (false when the encoder is unavailable or
-// rejects the tensor).
-bool tma_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows);
-// Records the persistent grid size that sba_attention_grid_size reports.
-void note_attention_grid_size(int grid);
 cudaError_t launch_smooth_v(const sba_plan* p, const void* vt, void* vq, float* vmean,
                             int32_t* vexp, void* workspace, cudaStream_t st);
 cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const void* kt, const void* vq,

@@ -63,19 +63,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test: has the phase of `bar` with parity `parity` completed?
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait for the phase of `bar` with parity `parity` to complete.
 // Polls try_wait; only every 1024 polls does it look at the CTA's abort flag
 // and at %globaltimer (whose read is slow, so it stays off the fast path).
@@ -151,33 +138,6 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
       : "memory");
-}
-
-// The same products with the accumulate flag fixed at compile time (no
-// predicate set-up between back-to-back issues).
-template <bool ACC>
-__device__ __forceinline__ void mma_ss_c(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
-  uint32_t z = 0;
-  if constexpr (ACC)
-    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%4, %4, %4, %4}, 1;" ::"r"(d_tmem),
-                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(z)
-                 : "memory");
-  else
-    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%4, %4, %4, %4}, 0;" ::"r"(d_tmem),
-                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(z)
-                 : "memory");
-}
-template <bool ACC>
-__device__ __forceinline__ void mma_ts_c(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
-  uint32_t z = 0;
-  if constexpr (ACC)
-    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%4, %4, %4, %4}, 1;" ::"r"(d_tmem),
-                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(z)
-                 : "memory");
-  else
-    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%4, %4, %4, %4}, 0;" ::"r"(d_tmem),
-                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(z)
-                 : "memory");
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]; A is K-major, one row per TMEM lane.
@@ -423,20 +383,6 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   p = ffma2(p, f, make_float2(0.99992806f, 0.99992806f));
   return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
-}
-
-// Register split between warpgroups (all four warps of a warpgroup execute
-// the same instruction): dec returns registers to the CTA's pool, inc waits
-// until the pool can grant the new count. The pool is the CTA's launch
-// allocation (threads x registers per thread at launch); the splits used
-// here fit in it.
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
