@@ -507,9 +507,16 @@ def stripe_mask(g: Geom, params, B: int) -> dict:
 #   removes it.
 # * Reference maximum: the row maximum of the first selected block; a later
 #   block whose maximum exceeds the reference by more than 2.75 (log2 units)
-#   replaces it (the accumulators are rescaled by 2^(old - new)), so that no
-#   code exceeds 126. With low-bit codes the reference changes the result, so
-#   this rule is part of the definition.
+#   replaces it (the accumulators are rescaled by 2^(old - new)); a block
+#   whose maximum lies exactly 2.75 above keeps it. The rule is forced by the
+#   online form the abstract gives (the mean comes back through the row sum
+#   that the online softmax keeps): codes are taken block by block, before
+#   later blocks are seen, against a reference that only moves forward, and
+#   2.75 is the headroom of the code range above the reference
+#   ((126 - 104) / 8), the largest jump that needs no rescale without a code
+#   clipping at 448. With low-bit codes the reference changes the codes (the
+#   fraction of 8x moves with it), so the rule, applied to the selected blocks
+#   in ascending key-block order, is part of the definition.
 
 E4M3_MAX = 448.0
 
@@ -592,16 +599,67 @@ def v_smooth_dequant(codes: np.ndarray, mu: np.ndarray, e: np.ndarray, g: Geom) 
     return np.where(valid[None, None, :, None], Vd, 0.0)
 
 
-def attention_fp8(Qt, Kt, codes, mu, e, g: Geom, row_ptr, col_idx, blocks=None):
+def expcast_reference(block_max, invert=None) -> np.ndarray:
+    """Reference maximum in force for each block of a row (reading above).
+
+    block_max [n, rows]: the rows' maxima over the real keys of their n
+    selected blocks, in col_idx order (log2 units). Returns [n, rows]: ref[0]
+    = block_max[0]; ref[k] = block_max[k] if block_max[k] > ref[k-1] + 2.75,
+    else ref[k-1]. ``invert`` (bool [n, rows]) takes the opposite decision at
+    the marked (block, row) pairs (block 0 has no decision): used to follow
+    a run that decided a near-threshold comparison the other way."""
+    bm = np.asarray(block_max, dtype=np.float64)
+    ref = np.empty_like(bm)
+    if bm.shape[0] == 0:
+        return ref
+    ref[0] = bm[0]
+    for k in range(1, bm.shape[0]):
+        replace = bm[k] > ref[k - 1] + EXPCAST_TAU
+        if invert is not None:
+            replace = replace ^ np.asarray(invert[k], dtype=bool)
+        ref[k] = np.where(replace, bm[k], ref[k - 1])
+    return ref
+
+
+# Margins of the rounding decisions. The oracle takes every decision of the
+# low-bit path in fp64 on exact scores; a run that forms the scores with fp32
+# accumulation (d products) and the code argument 8x + 104 with fp32 multiply-
+# adds can take a decision that lies within rounding distance of its boundary
+# the other way. The margin of a key's code argument (code units) is twice the
+# worst case of: the accumulation, d * 2^-23 * sum_i |q_i k_i| for the key and
+# for the reference's key, scaled by 8 * log2(e) / sqrt(d); the scale constant
+# and the product with it, 2^-23 * |8x| and 2^-22 * |8m|; the bias 104 - 8m
+# and the multiply-add, 2^-23 * 232. A replacement decision's margin (log2
+# units) is the largest key margin of its block over 8.
+def _fp8_margins(absdot, x, m, absdot_ref, c2, d):
+    acc = d * 2.0 ** -23 * (absdot + absdot_ref[:, None]) * 8.0 * c2
+    rnd = 2.0 ** -23 * np.abs(8.0 * x) + 2.0 ** -22 * np.abs(8.0 * m)[:, None] + 2.0 ** -23 * 232.0
+    return 2.0 * (acc + rnd)
+
+
+def attention_fp8(Qt, Kt, codes, mu, e, g: Geom, row_ptr, col_idx, blocks=None, invert=None,
+                  diag=False):
     """Block-sparse attention with ExpCast-FP8 probabilities and V-Smooth
     values (readings above), row by row in col_idx order.
 
-    Per selected block j of a row, on its real keys: x = q.k / sqrt(d) * log2(e)
-    - m, probabilities P = decode(expcast_code(x)), l_j = sum of P over the
+    Per selected block j of a row, on its real keys: x = q.k / sqrt(d) * log2(e),
+    references m from ``expcast_reference`` over the blocks' row maxima,
+    probabilities P = decode(expcast_code(x - m)), l_j = sum of P over the
     block; accumulators A += P @ (sigma * decode(codes_j)), L += l_j,
-    M += l_j * mu_j, all rescaled together when the reference m changes.
-    O = (A + M) / L, lse = ln(L) + (m - 6) * ln(2). Padding query slots:
-    O = 0, lse = 0. Returns (Ot, lse) like ``attention``."""
+    M += l_j * mu_j, all rescaled together by 2^(m_old - m_new) when the
+    reference moves. O = (A + M) / L, lse = ln(L) + (m - 6) * ln(2). Padding
+    query slots: O = 0, lse = 0. Returns (Ot, lse) like ``attention``.
+
+    ``invert``: {(b, h, i): bool [n, bs]} replacement decisions to take the
+    other way in that mask row (``expcast_reference``).
+    ``diag``: also return a dict of decision margins per query slot:
+    ``flip_o`` [B,H,Npad,d] and ``flip_lse`` [B,H,Npad], bounds on how far O
+    and lse move if every code whose argument lies within its margin of a
+    rounding boundary (k + 1/2, k = 0..125) takes the neighbouring code (the
+    probability moves by decode(k+1) - decode(k); O moves by that times
+    |v - O| over L, lse by -ln(1 - sum |dP| / L)); ``thr_near`` [B,H,Npad]
+    the number of replacement decisions within their margin of the threshold,
+    and ``thr_first`` [B,H,Npad] the block position of the first (-1: none)."""
     Qt = np.asarray(Qt, dtype=np.float64)
     Kt = np.asarray(Kt, dtype=np.float64)
     B, H, Npad, d = Qt.shape
@@ -610,6 +668,11 @@ def attention_fp8(Qt, Kt, codes, mu, e, g: Geom, row_ptr, col_idx, blocks=None):
     Vr = e4m3_decode(codes) * np.exp2(np.asarray(e, dtype=np.float64))[:, :, None, None]
     Ot = np.full((B, H, Npad, d), np.nan)
     lse = np.full((B, H, Npad), np.nan)
+    if diag:
+        flip_o = np.zeros((B, H, Npad, d))
+        flip_lse = np.zeros((B, H, Npad))
+        thr_near = np.zeros((B, H, Npad), dtype=np.int64)
+        thr_first = np.full((B, H, Npad), -1, dtype=np.int64)
     if blocks is None:
         blocks = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
     c2 = math.log2(math.e) / math.sqrt(d)
@@ -619,35 +682,81 @@ def attention_fp8(Qt, Kt, codes, mu, e, g: Geom, row_ptr, col_idx, blocks=None):
         q_slots = np.arange(i * bs, (i + 1) * bs)
         q = Qt[b, h, q_slots]
         n_q = q.shape[0]
+        keys = []
+        xs = []
+        for j in sel:
+            ks = np.arange(j * bs, (j + 1) * bs)
+            ks = ks[valid[ks]]
+            keys.append(ks)
+            xs.append((q @ Kt[b, h, ks].T) * c2)
+        if len(sel):
+            bmax = np.stack([x.max(axis=1) for x in xs])
+            ref = expcast_reference(bmax, None if invert is None else invert.get((b, h, i)))
         m = np.full(n_q, -np.inf)
         A = np.zeros((n_q, d))
         L = np.zeros(n_q)
         M = np.zeros((n_q, d))
+        F0 = np.zeros(n_q)       # sum of |dP| over near-boundary codes
+        F1 = np.zeros((n_q, d))  # sum of |dP| |v|
+        mkey = np.zeros(n_q)     # sum |q_i k_i| of the reference's key
         for idx, j in enumerate(sel):
-            ks = np.arange(j * bs, (j + 1) * bs)
-            ks = ks[valid[ks]]
-            x = (q @ Kt[b, h, ks].T) * c2
-            mblk = x.max(axis=1)
-            if idx == 0:
-                m_new = mblk
-            else:
-                m_new = np.where(mblk > m + EXPCAST_TAU, mblk, m)
+            x = xs[idx]
+            m_new = ref[idx]
             alpha = np.where(np.isfinite(m), np.exp2(np.where(np.isfinite(m), m - m_new, 0.0)), 0.0)
             A *= alpha[:, None]
             M *= alpha[:, None]
             L *= alpha
+            F0 *= alpha
+            F1 *= alpha[:, None]
+            if diag:
+                absdot = np.abs(q) @ np.abs(Kt[b, h, keys[idx]]).T
+                moved = m_new != m
+                arg = np.argmax(x, axis=1)
+                mkey = np.where(moved, absdot[np.arange(n_q), arg], mkey)
+                marg = _fp8_margins(absdot, x, m_new, mkey, c2, d)
+                if idx > 0:
+                    gap = np.abs(bmax[idx] - (m + EXPCAST_TAU))
+                    near = gap <= marg.max(axis=1) / 8.0
+                    rows = q_slots[near]
+                    thr_first[b, h, rows] = np.where(thr_first[b, h, rows] < 0, idx,
+                                                     thr_first[b, h, rows])
+                    thr_near[b, h, q_slots] += near
             m = m_new
+            y = 8.0 * (x - m[:, None]) + EXPCAST_BIAS
             P = e4m3_decode(expcast_code(x - m[:, None]))
             lj = P.sum(axis=1)
-            A += P @ Vr[b, h, ks]
+            vk = Vr[b, h, keys[idx]]
+            A += P @ vk
             M += lj[:, None] * mu[b, h, j].astype(np.float64)[None, :]
             L += lj
+            if diag:
+                kb = np.floor(y - 0.5)  # boundary k + 1/2 just below y
+                dist = np.minimum(np.abs(y - (kb + 0.5)), np.abs(y - (kb + 1.5)))
+                kk = np.where(np.abs(y - (kb + 0.5)) <= np.abs(y - (kb + 1.5)), kb, kb + 1)
+                hit = (dist <= marg) & (kk >= 0) & (kk <= 125)
+                kc = np.clip(kk, 0, 125).astype(np.int64)
+                dP = np.where(hit, e4m3_decode(kc + 1) - e4m3_decode(kc), 0.0)
+                vd = np.abs(vk + mu[b, h, j].astype(np.float64)[None, :])
+                F0 += dP.sum(axis=1)
+                F1 += dP @ vd
         qv = valid[q_slots]
         with np.errstate(divide="ignore", invalid="ignore"):
             o = (A + M) / L[:, None]
             ls = np.log(L) + (m - (EXPCAST_BIAS - 56.0) / 8.0) * math.log(2.0)
+            if diag:
+                den = np.maximum(L - F0, 0.0)
+                fo = np.where(F0[:, None] > 0, (F1 + np.abs(o) * F0[:, None]) / den[:, None], 0.0)
+                fl = np.where(F0 > 0, -np.log(np.maximum(1.0 - F0 / L, 1e-300)), 0.0)
         o[~qv] = 0.0
         ls[~qv] = 0.0
         Ot[b, h, q_slots] = o
         lse[b, h, q_slots] = ls
+        if diag:
+            fo[~qv] = 0.0
+            fl[~qv] = 0.0
+            flip_o[b, h, q_slots] = fo
+            flip_lse[b, h, q_slots] = fl
+    if diag:
+        return Ot, lse, {"flip_o": flip_o, "flip_lse": flip_lse, "thr_near": thr_near,
+                         "thr_first": thr_first}
     return Ot, lse

@@ -757,3 +757,153 @@ def test_fp8_reference_max_is_replaced_when_a_later_block_dominates():
                                 blocks=[(0, 0, 0)])
     sl = slice(0, g.bs)
     assert np.allclose(O8[0, 0, sl], only2[0, 0, sl], atol=1e-4)
+
+
+# Reference rule of ExpCast-FP8 (VC-Attention abstract: codes from one
+# multiply-add inside the online softmax). Hand-worked rows: block maxima in
+# log2 units, in col_idx order, and the reference in force at each block.
+_REFERENCE_ROWS = [
+    ([0.0, 2.70, 2.80], [0.0, 0.0, 2.80]),    # 2.70 keeps; 2.80 is more than 2.75 above 0
+    ([0.0, 2.75], [0.0, 0.0]),                # exactly 2.75 above keeps (strict >)
+    ([0.0, 2.70, 5.50], [0.0, 0.0, 5.50]),
+    ([1.0, -3.0, 3.76, 3.70], [1.0, 1.0, 3.76, 3.76]),
+    ([1.0, 3.74, 6.5, 9.2501], [1.0, 1.0, 6.5, 9.2501]),
+    ([-4.0, -9.0, -1.25, -1.2499], [-4.0, -4.0, -4.0, -1.2499]),
+]
+
+
+def _reference_pins_hold(rule) -> bool:
+    for bm, want in _REFERENCE_ROWS:
+        got = rule(np.array(bm)[:, None])[:, 0]
+        if not np.array_equal(got, np.array(want)):
+            return False
+    return True
+
+
+def test_expcast_reference_hand_worked_rows():
+    assert _reference_pins_hold(_o.expcast_reference)
+    # invert takes the other decision at the marked block only
+    inv = np.zeros((3, 1), dtype=bool)
+    inv[1, 0] = True
+    assert _o.expcast_reference(np.array([[0.0], [2.70], [2.80]]), inv)[:, 0].tolist() == \
+        [0.0, 2.70, 2.70]
+
+
+def test_expcast_reference_pins_catch_plausible_slips():
+    """The pins fail for a >= comparison and for a rule that compares with
+    the running maximum instead of the reference."""
+    def ge_rule(bm):
+        ref = np.empty_like(bm)
+        ref[0] = bm[0]
+        for k in range(1, len(bm)):
+            ref[k] = np.where(bm[k] >= ref[k - 1] + 2.75, bm[k], ref[k - 1])
+        return ref
+
+    def running_max_rule(bm):
+        ref = np.empty_like(bm)
+        ref[0] = bm[0]
+        run = bm[0].copy()
+        for k in range(1, len(bm)):
+            ref[k] = np.where(bm[k] > run + 2.75, bm[k], ref[k - 1])
+            run = np.maximum(run, bm[k])
+        return ref
+
+    assert not _reference_pins_hold(ge_rule)
+    assert not _reference_pins_hold(running_max_rule)
+
+
+def _one_row_case(xs, vals, d=8):
+    """One mask row over blocks 0..len(xs)-1 of a 4-block layer of 64-token
+    cubes: every key of block j scores xs[j] (log2 units) against every query,
+    and every value of block j is vals[j] (so V-Smooth stores zero codes and
+    the block means carry the values)."""
+    g = Geom(4, 8, 8, 4, 4, 4)
+    c2 = math.log2(math.e) / math.sqrt(d)
+    Qt = np.zeros((1, 1, g.Npad, d))
+    Qt[..., 0] = 1.0
+    Kt = np.zeros((1, 1, g.Npad, d))
+    Vt = np.zeros((1, 1, g.Npad, d))
+    for j, (x, v) in enumerate(zip(xs, vals)):
+        Kt[0, 0, j * g.bs:(j + 1) * g.bs, 0] = x / c2
+        Vt[0, 0, j * g.bs:(j + 1) * g.bs] = v
+    codes, mu, e = _o.v_smooth(Vt, g)
+    assert not codes.any()
+    n = len(xs)
+    rp = np.array([0] + [n] * g.nb)
+    ci = np.arange(n)
+    return g, Qt, Kt, codes, mu, e, rp, ci
+
+
+@pytest.mark.parametrize("xs,refs", [([0.0, 2.70, 2.80], [2.80, 2.80, 2.80]),
+                                     ([0.0, 2.70, 5.50], [5.50, 5.50, 5.50]),
+                                     ([0.0, -2.0, 2.70], [0.0, 0.0, 0.0])])
+def test_fp8_attention_hand_worked_reference_rows(xs, refs):
+    """O and lse of one row worked by hand from the code table: a block at x
+    (log2 units) against the reference it is coded under (its own m at the
+    time) takes code rint(8(x - m) + 104), and the accumulators carry a factor
+    2^(m - m_final) for every later replacement."""
+    vals = [np.full(8, 1.0), np.full(8, -2.0), np.full(8, 5.0)]
+    g, Qt, Kt, codes, mu, e, rp, ci = _one_row_case(xs, vals)
+    m_at = _o.expcast_reference(np.array(xs)[:, None])[:, 0]
+    # codes by hand: 104 at the reference, 8 * 2.70 + 104 = 125.6 -> 126 (448),
+    # 8 * -2 + 104 = 88 (16)
+    table = {104: 64.0, 126: 448.0, 88: 16.0}
+    w = []
+    for x, m in zip(xs, m_at):
+        c = int(round(8 * (x - m) + 104))
+        w.append(64 * table[c] * 2.0 ** (m - refs[-1]))
+    L = sum(w)
+    want_o = sum(wi * v for wi, v in zip(w, vals)) / L
+    want_lse = math.log(L) + (refs[-1] - 6.0) * math.log(2.0)
+    O8, l8 = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci, blocks=[(0, 0, 0)])
+    assert np.allclose(O8[0, 0, :g.bs], want_o, rtol=1e-12, atol=1e-12)
+    assert np.allclose(l8[0, 0, :g.bs], want_lse, rtol=1e-12, atol=1e-12)
+    assert list(m_at) == [0.0, 0.0, refs[-1]] or xs[-1] < 2.75
+
+
+def test_fp8_flip_bound_covers_a_code_on_its_rounding_boundary():
+    """Block 1 scores sit on the boundary between codes 95 and 96
+    (8 * -1.0625 + 104 = 95.5): nudging them either way flips all 64 codes.
+    The margin report flags them, its bound covers the actual move of O and
+    lse, and is within a small factor of it."""
+    vals = [np.full(8, 1.0), np.full(8, -2.0)]
+    outs = []
+    for eps in (1e-9, -1e-9):
+        g, Qt, Kt, codes, mu, e, rp, ci = _one_row_case([0.0, -1.0625 + eps], vals)
+        O8, l8, dg = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci, blocks=[(0, 0, 0)], diag=True)
+        outs.append((O8[0, 0, 0], l8[0, 0, 0], dg["flip_o"][0, 0, 0], dg["flip_lse"][0, 0, 0],
+                     dg["thr_near"][0, 0, 0]))
+    (o1, l1, f1, fl1, t1), (o2, l2, f2, fl2, t2) = outs
+    move = np.abs(o1 - o2)
+    assert move.min() > 1e-3                       # the flip is real
+    assert np.all(move <= f1) and np.all(move <= f2)
+    assert np.all(f1 <= 3.0 * move) and np.all(f2 <= 3.0 * move)
+    # (the lse bound is exact for a flip that lowers the sum: equal up to rounding)
+    assert abs(l1 - l2) <= min(fl1, fl2) + 1e-12 and max(fl1, fl2) <= 3.0 * abs(l1 - l2)
+    assert t1 == 0 and t2 == 0
+    # away from any boundary the report is empty
+    g, Qt, Kt, codes, mu, e, rp, ci = _one_row_case([0.0, -1.0], vals)
+    _, _, dg = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci, blocks=[(0, 0, 0)], diag=True)
+    assert not dg["flip_o"].any() and not dg["flip_lse"].any()
+
+
+def test_fp8_threshold_report_and_the_other_decision():
+    """A block maximum exactly 2.75 above the reference is flagged; the
+    inverted decision reproduces a run that replaced the reference there."""
+    vals = [np.full(8, 1.0), np.full(8, -2.0)]
+    g, Qt, Kt, codes, mu, e, rp, ci = _one_row_case([0.0, 2.75], vals)
+    O8, l8, dg = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci, blocks=[(0, 0, 0)], diag=True)
+    assert np.all(dg["thr_near"][0, 0, :g.bs] == 1) and np.all(dg["thr_first"][0, 0, :g.bs] == 1)
+    inv = np.zeros((2, g.bs), dtype=bool)
+    inv[1] = True
+    Oi, li = _o.attention_fp8(Qt, Kt, codes, mu, e, g, rp, ci, blocks=[(0, 0, 0)],
+                              invert={(0, 0, 0): inv})
+    # by hand: kept -> codes 104 and 126 (64, 448); replaced -> block 0 keeps
+    # the code it took under the old reference (104: 64), rescaled by
+    # 2^(0 - 2.75), and block 1 takes 104 (64)
+    w0 = 64.0 * 2.0 ** -2.75
+    kept = (64 * 1.0 + 448 * -2.0) / (64 + 448)
+    repl = (w0 * 1.0 + 64 * -2.0) / (w0 + 64)
+    assert np.allclose(O8[0, 0, 0], kept, atol=1e-12)
+    assert np.allclose(Oi[0, 0, 0], repl, atol=1e-12)
+    assert np.isclose(li[0, 0, 0], math.log(64 * (w0 + 64)) + (2.75 - 6.0) * math.log(2.0))
