@@ -294,9 +294,15 @@ class Plan:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
+        if not h:
+            return
+        self.handle = None
+        try:
             sba_plan_destroy(h)
-            self.handle = None
+        except (TypeError, AttributeError):
+            # interpreter shutdown: the module's globals are already cleared
+            # and the process releases the library with everything else
+            pass
 
 
 class SparseAttention:

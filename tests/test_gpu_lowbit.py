@@ -4,15 +4,19 @@ through the C ABI.
 
 sba_smooth_v is integer work once its fp32 inputs are fixed: codes, block
 means and exponents are compared bit-exactly with the oracle on the GPU's own
-reordered values. sba_attention_lowbit is compared with the oracle's low-bit
-attention on the GPU's CSR and codes: rel-L2 <= 1e-2 as for bf16, and
-element-wise within 2e-2 (lse within 1e-2) except for rare outputs that a single
-probability code decided differently: the kernel rounds 8x + 104 from fp32
-tensor-core scores, the oracle from fp64 scores, so at a rounding boundary the
-two take adjacent codes (values up to 12.5 % apart); if that key dominates its
-row the output moves by up to ~0.1. Such outputs must be under 0.1 % of all
-and within 0.15. The departure from exact attention is the quantisation error
-of the method and is only bounded loosely (rel-L2 < 6 %)."""
+reordered values. sba_attention_lowbit is compared with the oracle's low-bit attention on the
+GPU's CSR and codes: rel-L2 <= 1e-2 as for bf16, and every output within 2e-2
+(lse within 1e-2) plus the oracle's own bound on what codes near a rounding
+boundary can change. The kernel rounds 8x + 104 from fp32 tensor-core scores,
+the oracle from fp64 scores; a code whose argument lies within rounding
+distance of k + 1/2 may come out as the neighbouring code, and the oracle
+reports, per query row, how far O and lse can move if all such codes flip. A
+query row with a reference-replacement decision within rounding distance of
+its threshold is checked against the oracle run that takes that decision the
+other way as well (either must match); a row with two such decisions is
+exempt and counted. The departure from exact attention is the quantisation
+error of the method and is only bounded loosely (rel-L2 < 6 %).
+"""
 import math
 
 import numpy as np
@@ -67,40 +71,69 @@ def _check_smooth(wl, gpu):
 def _check_attention(wl, gpu, codes, mu, e, blocks):
     g = geom_of(wl)
     valid = oracle.slot_valid(g)
-    ref_rows, got_rows, ref_l, got_l, ex_rows = [], [], [], [], []
+    ref_rows, got_rows, ref_l, got_l, ex_rows, fo_rows, fl_rows = [], [], [], [], [], [], []
     by_head = {}
     for (b, h, i) in blocks:
         by_head.setdefault((b, h), []).append(i)
+    n_thr = n_exempt = n_flip_rows = 0
     for (b, h), idx in by_head.items():
         base = (b * wl.H + h) * g.nb
         rp = gpu["row_ptr"][base:base + g.nb + 1] - gpu["row_ptr"][base]
         ci = gpu["col_idx"][gpu["row_ptr"][base]:gpu["row_ptr"][base + g.nb]]
         qt = to64(gpu["qt"][b:b + 1, h:h + 1])
         kt = to64(gpu["kt"][b:b + 1, h:h + 1])
-        Ot, lse = oracle.attention_fp8(qt, kt, codes[b:b + 1, h:h + 1], mu[b:b + 1, h:h + 1],
-                                       e[b:b + 1, h:h + 1], g, rp, ci, blocks=[(0, 0, i) for i in idx])
+        args = (qt, kt, codes[b:b + 1, h:h + 1], mu[b:b + 1, h:h + 1], e[b:b + 1, h:h + 1], g, rp, ci)
+        Ot, lse, dg = oracle.attention_fp8(*args, blocks=[(0, 0, i) for i in idx], diag=True)
         Ox, _ = oracle.attention(qt, kt, to64(gpu["vt"][b:b + 1, h:h + 1]), g, rp, ci,
                                  blocks=[(0, 0, i) for i in idx])
         for i in idx:
             sl = slice(i * g.bs, (i + 1) * g.bs)
-            m = valid[sl]
-            ref_rows.append(Ot[0, 0, sl][m])
+            m = valid[sl].copy()
+            got_o = to64(gpu["ot"][b, h, sl])
+            got_lse = gpu["lse"][b, h, sl].double().numpy()
+            o_ref, l_ref = Ot[0, 0, sl].copy(), lse[0, 0, sl].copy()
+            fo, fl = dg["flip_o"][0, 0, sl], dg["flip_lse"][0, 0, sl]
+            near = dg["thr_near"][0, 0, sl]
+            n_thr += int((near[m] > 0).sum())
+            n_flip_rows += int((fo.max(axis=1)[m] > 0).sum())
+            one = m & (near == 1)
+            if one.any():
+                # the other decision at the flagged block, for those query rows
+                inv = np.zeros((rp[i + 1] - rp[i], g.bs), dtype=bool)
+                inv[dg["thr_first"][0, 0, sl][one], np.nonzero(one)[0]] = True
+                Oa, la, dga = oracle.attention_fp8(*args, blocks=[(0, 0, i)], invert={(0, 0, i): inv},
+                                                   diag=True)
+                for q in np.nonzero(one)[0]:
+                    fits = lambda o, l, f, fl_: (np.all(np.abs(got_o[q] - o) <= ATOL + f) and
+                                                 abs(got_lse[q] - l) <= 1e-2 + fl_)
+                    if not fits(o_ref[q], l_ref[q], fo[q], fl[q]):
+                        o_ref[q], l_ref[q] = Oa[0, 0, sl][q], la[0, 0, sl][q]
+                        fo[q], fl[q] = dga["flip_o"][0, 0, sl][q], dga["flip_lse"][0, 0, sl][q]
+            two = m & (near >= 2)
+            n_exempt += int(two.sum())
+            m &= ~two
+            ref_rows.append(o_ref[m])
             ex_rows.append(Ox[0, 0, sl][m])
-            got_rows.append(to64(gpu["ot"][b, h, sl])[m])
-            ref_l.append(lse[0, 0, sl][m])
-            got_l.append(gpu["lse"][b, h, sl].double().numpy()[m])
+            got_rows.append(got_o[m])
+            ref_l.append(l_ref[m])
+            got_l.append(got_lse[m])
+            fo_rows.append(fo[m])
+            fl_rows.append(fl[m])
     R, G, X = np.concatenate(ref_rows), np.concatenate(got_rows), np.concatenate(ex_rows)
+    FO, FL = np.concatenate(fo_rows), np.concatenate(fl_rows)
     mx, rel = attention_errors(G, R)
     err = np.abs(G - R)
-    frac = float((err > ATOL).mean())
-    worst = np.unravel_index(int(np.argmax(err)), err.shape)
-    info = (mx, rel, frac, worst)
+    worst = np.unravel_index(int(np.argmax(err - FO)), err.shape)
+    info = (mx, rel, worst, float(err[worst]), float(FO[worst]))
+    beyond = int((err > ATOL).sum())
+    print(f"query rows {R.shape[0]}: with near-boundary codes {n_flip_rows}, near-threshold "
+          f"{n_thr}, exempt {n_exempt}; max |err| {mx:.3g}, outputs beyond {ATOL} {beyond} "
+          f"(of {err.size}), median flip bound {float(np.median(FO)):.2g}")
     assert rel <= REL_L2, info
-    assert frac <= 1e-3 and mx <= 0.15, info
-    # lse: a flipped code moves the row's denominator by up to 12.5 % of that
-    # key's share, i.e. lse by up to ln(1.125)
+    assert np.all(err <= ATOL + FO), info
     dl = np.abs(np.concatenate(got_l) - np.concatenate(ref_l))
-    assert float((dl > 1e-2).mean()) <= 1e-3 and dl.max() <= math.log(1.125), (dl.max(),)
+    assert np.all(dl <= 1e-2 + FL), (dl.max(),)
+    assert n_exempt <= max(2, R.shape[0] // 1000), n_exempt
     _, rel_exact = attention_errors(G, X)
     assert rel_exact < 0.06, rel_exact
     return mx, rel, rel_exact
