@@ -39,7 +39,8 @@ SBA_ORDER_HILBERT = 1
 
 EXPORTED = ["sba_plan_create", "sba_plan_destroy", "sba_plan_query", "sba_workspace_init",
             "sba_reorder", "sba_unreorder", "sba_build_mask", "sba_attention",
-            "sba_check_device_status", "sba_debug_timeout_probe", "sba_perm_export",
+            "sba_check_device_status", "sba_debug_timeout_probe", "sba_debug_exp2_poly",
+            "sba_perm_export",
             "sba_attention_grid_size", "sba_status_string", "sba_last_error",
             "sba_build_mask_noalloc", "sba_build_stripe_mask", "sba_smooth_v",
             "sba_attention_lowbit", "sba_noalloc_status"]
@@ -86,6 +87,7 @@ _sig = {
     "sba_check_device_status": [_vp, _vp, _vp],
     "sba_noalloc_status": [_vp],
     "sba_debug_timeout_probe": [_vp, _vp, ctypes.c_uint64, _vp],
+    "sba_debug_exp2_poly": [_vp, _vp, ctypes.c_int64, _vp],
     "sba_perm_export": [_vp, ctypes.POINTER(ctypes.c_int32)],
     "sba_attention_grid_size": [],
     "sba_status_string": [_i32],
@@ -236,6 +238,16 @@ def sba_noalloc_status(stream=None) -> int:
 def sba_check_device_status(plan: int, workspace, stream=None) -> int:
     """Returns the status code (does not raise on device-side errors)."""
     return _lib.sba_check_device_status(plan, _ptr(workspace), _stream(stream))
+
+
+def sba_debug_exp2_poly(x, y, stream=None) -> None:
+    """y = 2^x through the attention softmax's FMA-pipe exponential (fp32
+    device tensors of equal length)."""
+    import torch
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise SbaError(SBA_ERR_INVALID_ARG, "x and y must be fp32 tensors of equal length")
+    _check(_lib.sba_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "sba_debug_exp2_poly")
 
 
 def sba_debug_timeout_probe(plan: int, workspace, timeout_ns: int, stream=None) -> None:

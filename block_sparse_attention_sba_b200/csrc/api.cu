@@ -195,12 +195,19 @@ sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
   p->ws_qbar = 256;
   const size_t pooled = align256(static_cast<size_t>(R) * G.d * sizeof(double));
   p->ws_kbar = p->ws_qbar + pooled;
-  p->ws_perm = p->ws_kbar + pooled;
+  // pooled scores: all heads, or as many as 48 MiB hold (at least one)
+  const size_t per_head = static_cast<size_t>(nb) * nb * sizeof(double);
+  const size_t all_heads = per_head * static_cast<size_t>(G.B) * G.H;
+  p->scores_bytes = std::min(all_heads, std::max(per_head, size_t(48) << 20) / per_head * per_head);
+  p->ws_scores = p->ws_kbar + pooled;
+  p->ws_perm = p->ws_scores + align256(p->scores_bytes);
   p->info.workspace_bytes = p->ws_perm;
   if (G.order == SBA_ORDER_HILBERT) {
     build_hilbert_tables(p);
     p->info.workspace_bytes += align256(static_cast<size_t>(Npad) * sizeof(int32_t));
   }
+  p->ws_heads = p->info.workspace_bytes;
+  p->info.workspace_bytes += align256(static_cast<size_t>(G.B) * G.H * sizeof(uint32_t));
   p->wait_budget_ns = 4000000000ull;  // 4 s: no healthy wait comes near it
   const char* env = getenv("SBA_WAIT_BUDGET_NS");
   if (env) {
@@ -224,6 +231,9 @@ sba_status sba_workspace_init(const sba_plan* plan, void* workspace, void* strea
   if (!plan || !workspace) return fail(SBA_ERR_INVALID_ARG, "plan and workspace must be non-NULL");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(Ctrl), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  e = cudaMemsetAsync(static_cast<char*>(workspace) + plan->ws_heads, 0,
+                      static_cast<size_t>(plan->g.B) * plan->g.H * sizeof(uint32_t), st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   if (plan->g.order == SBA_ORDER_HILBERT) {
     // from pageable host memory: returns once the table has been staged
@@ -291,7 +301,8 @@ sba_status sba_build_mask(const sba_plan* plan, const void* qt, const void* kt, 
   cudaError_t e = launch_build_mask(plan, qt, kt, top_p, top_k, bitmask, row_cnt, row_ptr, col_idx,
                                     work_order, reinterpret_cast<double*>(ws + plan->ws_qbar),
                                     reinterpret_cast<double*>(ws + plan->ws_kbar),
-                                    &reinterpret_cast<Ctrl*>(ws + plan->ws_ctrl)->status,
+                                    reinterpret_cast<double*>(ws + plan->ws_scores), plan->scores_bytes,
+                                    reinterpret_cast<Ctrl*>(ws + plan->ws_ctrl),
                                     static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "sba_build_mask launch");
 }
@@ -394,6 +405,15 @@ sba_status sba_debug_timeout_probe(const sba_plan* plan, void* workspace, uint64
     return fail(SBA_ERR_INVALID_ARG, "timeout_ns must lie in [1e3, 1e10]");
   cudaError_t e = launch_timeout_probe(workspace, timeout_ns, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SBA_OK : cuda_fail(e, "timeout probe launch");
+}
+
+sba_status sba_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  g_err[0] = '\0';
+  if (n < 0 || n > (int64_t(1) << 31)) return fail(SBA_ERR_INVALID_ARG, "n must lie in [0, 2^31]");
+  if (n == 0) return SBA_OK;
+  if (!x || !y) return fail(SBA_ERR_INVALID_ARG, "x and y must be non-NULL");
+  cudaError_t e = launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBA_OK : cuda_fail(e, "exp2 polynomial launch");
 }
 
 sba_status sba_perm_export(const sba_plan* plan, int32_t* slot_of_token) {

@@ -93,11 +93,13 @@ struct Cfg {
   // codes have 2.75 octaves of headroom above the reference (code 104 of 126).
   static constexpr float RESCALE = LB ? 2.75f : 24.0f;
   static constexpr float LB_BIAS = 104.0f;  // E4M3 code of the reference
+  // bs = 64: a work item is a pair of query blocks (2i, 2i+1) of one head,
+  // whose 128 rows fill the tile, over the union of their key sets
+  static constexpr bool PAIR = BS == 64 && !LB;
   static_assert(!LB || (D == 128 && BS == 128), "low-bit path: d = bs = 128");
   // Request at least 120 KB so that only one CTA (one 512-column TMEM
   // allocation) is ever resident per SM.
   static constexpr int SMEM = SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED;
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(M, BS, 0, 0);
   static constexpr uint32_t IDESC_PV = LB ? idesc_e4m3_f32(M, D) : idesc_bf16_f32(M, D, 0, 1);
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_O = 384;
@@ -138,6 +140,21 @@ struct AttnParams {
 // integer (nearest even) held in the low mantissa bits.
 constexpr float kCodeMagic = 12582912.0f;
 
+// Next block of the ascending union of two sorted column lists (a pair's two
+// mask rows): returns it and whether each row selects it. Past both ends it
+// returns INT_MAX (only when the lists are inconsistent with the count).
+__device__ __forceinline__ int union_next(const int32_t* __restrict__ col_idx, int& ia, int nA, int sA,
+                                          int& ib, int nB, int sB, bool& inA, bool& inB) {
+  const int a = ia < nA ? __ldg(&col_idx[sA + ia]) : 0x7fffffff;
+  const int b = ib < nB ? __ldg(&col_idx[sB + ib]) : 0x7fffffff;
+  const int j = min(a, b);
+  inA = a == j;
+  inB = b == j;
+  ia += inA ? 1 : 0;
+  ib += inB ? 1 : 0;
+  return j;
+}
+
 // Wait that ignores the abort flag (used to drain in-flight async work).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t budget_ns,
                                                 uint32_t* status) {
@@ -161,11 +178,13 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(ctl);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 512);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 516);
-  int* ring = reinterpret_cast<int*>(ctl + 528);             // [2][4]
+  // work item ring [2][8]: item, blocks, start, n (row or first row of a
+  // pair), start and n of a pair's second row
+  int* ring = reinterpret_cast<int*>(ctl + 528);
   // real keys of the block each K / V slot holds (written before the slot's
   // TMA arrive, read after its full barrier)
-  int* klen_k = reinterpret_cast<int*>(ctl + 576);  // [NK]
-  int* klen_v = reinterpret_cast<int*>(ctl + 640);  // [NV]
+  int* klen_k = reinterpret_cast<int*>(ctl + 640);  // [NK]
+  int* klen_v = reinterpret_cast<int*>(ctl + 704);  // [NV]
   float* xmax = reinterpret_cast<float*>(ctl + 1024);        // [NSB][NWG][128] partial row maxima
   float* xsum = xmax + C::NSB * C::NWG * 128;                // [NWG][128] partial row sums
 
@@ -235,7 +254,8 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
         if (lane == 0) idx = static_cast<int>(atomicAdd(&P.ctrl->work_next, 1u));
         idx = __shfl_sync(0xffffffffu, idx, 0);
         if (idx < P.R) {
-          row = __ldg(&P.work_order[idx]);
+          // pairs are taken in order (the work order ranks mask rows)
+          row = C::PAIR ? idx : __ldg(&P.work_order[idx]);
           if (row < 0 || row >= P.R) {
             if (lane == 0) atomicOr(status, kStatusCheck);
             row = -1;
@@ -244,15 +264,43 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       } else {
         row = (items == 0) ? static_cast<int>(blockIdx.x) : -1;
       }
-      int start = 0, n = 0;
-      if (row >= 0) {
-        start = __ldg(&P.row_ptr[row]);
-        n = __ldg(&P.row_ptr[row + 1]) - start;
-        if (n < 0 || n > g.nb || start < 0 || static_cast<int64_t>(start) + n > P.max_nnz) {
-          // a row that cannot be read is skipped (written as empty)
+      // a mask row's selected blocks; a row that cannot be read is skipped
+      // (written as empty)
+      auto row_range = [&](int r, int& st0, int& cnt) {
+        st0 = __ldg(&P.row_ptr[r]);
+        cnt = __ldg(&P.row_ptr[r + 1]) - st0;
+        if (cnt < 0 || cnt > g.nb || st0 < 0 || static_cast<int64_t>(st0) + cnt > P.max_nnz) {
           if (lane == 0) atomicOr(status, kStatusCheck);
-          n = 0;
-          start = 0;
+          cnt = 0;
+          st0 = 0;
+        }
+      };
+      int start = 0, n = 0, nA = 0, startB = 0, nB = 0;
+      if (row >= 0) {
+        if constexpr (C::PAIR) {
+          // item = pair index; rows 2i and 2i+1 (if it exists) of head bh
+          const int hp = (g.nb + 1) >> 1;
+          const int bhp = row / hp, ip = row - bhp * hp;
+          const int rA = bhp * g.nb + 2 * ip;
+          row_range(rA, start, nA);
+          if (2 * ip + 1 < g.nb) row_range(rA + 1, startB, nB);
+          // union size = nA + nB - |A and B| (binary search of A's blocks in B)
+          int inter = 0;
+          for (int a = lane; a < nA; a += 32) {
+            const int x = __ldg(&P.col_idx[start + a]);
+            int lo = 0, hi = nB;
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (__ldg(&P.col_idx[startB + mid]) < x) lo = mid + 1; else hi = mid;
+            }
+            inter += (lo < nB && __ldg(&P.col_idx[startB + lo]) == x) ? 1 : 0;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) inter += __shfl_xor_sync(0xffffffffu, inter, o);
+          n = nA + nB - inter;
+        } else {
+          row_range(row, start, n);
+          nA = n;
         }
       }
       const int rs = items & 1;
@@ -261,16 +309,25 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
         if (!ok) break;
       }
       if (lane == 0) {
-        ring[rs * 4 + 0] = row;
-        ring[rs * 4 + 1] = n;
-        ring[rs * 4 + 2] = start;
+        ring[rs * 8 + 0] = row;
+        ring[rs * 8 + 1] = n;
+        ring[rs * 8 + 2] = start;
+        ring[rs * 8 + 3] = nA;
+        ring[rs * 8 + 4] = startB;
+        ring[rs * 8 + 5] = nB;
         mbar_arrive(bar(C::B_IF + rs));
       }
       ++items;
       if (row < 0) break;
       if (n == 0) continue;
       uint32_t bh, iq;
-      g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
+      if constexpr (C::PAIR) {
+        const int hp = (g.nb + 1) >> 1;
+        bh = static_cast<uint32_t>(row / hp);
+        iq = static_cast<uint32_t>(2 * (row - static_cast<int>(bh) * hp));
+      } else {
+        g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
+      }
       const int rows_base = static_cast<int>(bh) * g.Npad;
       if (qloads >= 1) {
         ok = wait1(C::B_QE, (qloads - 1) & 1);
@@ -286,12 +343,18 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       // K runs up to NSB-1 blocks ahead of V (the S issuer works that far ahead)
       int nk = 0, nv = 0;
       int ck = 0, cv = 0, ckb = -32, cvb = -32;
+      int iaK = 0, ibK = 0, iaV = 0, ibV = 0;  // pair: union cursors of K and V
       while (nv < n) {
         const bool isv = !(nk < n && nk <= nv + (C::NSB - 1));
         const int blk = isv ? nv : nk;
         const int cb = blk & ~31;
         int j;
-        if (!isv) {
+        if constexpr (C::PAIR) {
+          bool inA, inB;
+          j = isv ? union_next(P.col_idx, iaV, nA, start, ibV, nB, startB, inA, inB)
+                  : union_next(P.col_idx, iaK, nA, start, ibK, nB, startB, inA, inB);
+          (void)cb;
+        } else if (!isv) {
           if (cb != ckb) {
             ckb = cb;
             ck = (cb + lane < n) ? __ldg(&P.col_idx[start + cb + lane]) : 0;
@@ -386,7 +449,7 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       const int rs = items & 1;
       ok = wait1(C::B_IF + rs, (items >> 1) & 1);
       if (!ok) break;
-      const int row = ring[rs * 4 + 0], n = ring[rs * 4 + 1];
+      const int row = ring[rs * 8 + 0], n = ring[rs * 8 + 1];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_IE + rs));
       ++items;
@@ -440,7 +503,7 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       const int rs = items & 1;
       ok = wait1(C::B_IF + rs, (items >> 1) & 1);
       if (!ok) break;
-      const int row = ring[rs * 4 + 0], n = ring[rs * 4 + 1];
+      const int row = ring[rs * 8 + 0], n = ring[rs * 8 + 1];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_IE + rs));
       ++items;
@@ -521,20 +584,34 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       const int rs = items & 1;
       ok = wwait(C::B_IF + rs, (items >> 1) & 1);
       if (!ok) break;
-      const int row = ring[rs * 4 + 0], n = ring[rs * 4 + 1], start = ring[rs * 4 + 2];
+      const int row = ring[rs * 8 + 0], n = ring[rs * 8 + 1], start = ring[rs * 8 + 2];
+      const int nA = ring[rs * 8 + 3], startB = ring[rs * 8 + 4], nB = ring[rs * 8 + 5];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_IE + rs));
       ++items;
       if (row < 0) break;
       const uint64_t t_start = globaltimer_ns();
       uint32_t bh, iq;
-      g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
+      // pair items: rows t < 64 belong to query block iq, rows t >= 64 to
+      // block iq + 1 (written only when it exists); otherwise rows t < BS
+      bool has_rows = t < BS;
+      if constexpr (C::PAIR) {
+        const int hp = (g.nb + 1) >> 1;
+        bh = static_cast<uint32_t>(row / hp);
+        iq = static_cast<uint32_t>(2 * (row - static_cast<int>(bh) * hp));
+        has_rows = t < BS || static_cast<int>(iq) + 1 < g.nb;
+      } else {
+        g.dv_nb.divmod(static_cast<uint32_t>(row), bh, iq);
+      }
       // a block's real slots are its first block_len slots
-      const bool qvalid = t < block_len(g, static_cast<int>(iq));
+      const bool qvalid = has_rows && (t < BS ? t < block_len(g, static_cast<int>(iq))
+                                              : t - BS < block_len(g, static_cast<int>(iq) + 1));
       const int64_t orow = static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(iq) * BS + t;
       __nv_bfloat16* optr = P.ot + orow * D + wg * DPW;
+      // pair items: this warp's rows belong to the first (A) or second (B) row
+      const bool half_b = C::PAIR && (warp & 3) >= 2;
       if (n == 0) {
-        if (t < BS) {
+        if (has_rows) {
           for (int c = 0; c < DPW; c += 8)
             *reinterpret_cast<uint4*>(optr + c) = make_uint4(0u, 0u, 0u, 0u);
           if (P.lse && wg == 0) P.lse[orow] = qvalid ? -INFINITY : 0.f;
@@ -542,15 +619,45 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
       } else {
         float m = -INFINITY, l = 0.f;  // l: this group's share of the row sum
         int jn = __ldg(&P.col_idx[start]);
+        int ia = 0, ib = 0;  // pair: union cursors
         for (int i = 0; i < n; ++i) {
-          const int j = (jn < 0 || jn >= g.nb) ? 0 : jn;
-          if (i + 1 < n) jn = __ldg(&P.col_idx[start + i + 1]);
+          int j;
+          bool sel = true;  // this warp's rows select the block
+          if constexpr (C::PAIR) {
+            bool inA, inB;
+            j = union_next(P.col_idx, ia, nA, start, ib, nB, startB, inA, inB);
+            sel = half_b ? inB : inA;
+            if (j < 0 || j >= g.nb) j = 0;
+          } else {
+            j = (jn < 0 || jn >= g.nb) ? 0 : jn;
+            if (i + 1 < n) jn = __ldg(&P.col_idx[start + i + 1]);
+          }
           const int b = static_cast<int>(gsm % NSB);
           const uint32_t ph = (gsm / NSB) & 1;
           ok = wwait(C::B_SR + b, ph);
           if (!ok) break;
           tc_fence_after();
           const uint32_t scol = tmem + lane_off + static_cast<uint32_t>(b) * 128u;
+          if (C::PAIR && !sel) {
+            // rows that do not select the block: P = 0 over this group's
+            // columns, no maximum (-inf in the exchange), nothing added
+            float* xm0 = xmax + (b * NWG) * 128;
+            xm0[wg * 128 + t] = -INFINITY;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_X + b));
+            uint32_t zero[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) zero[e] = 0u;
+            tmem_st16(scol + wg * (CPW / 2), zero);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(C::B_PR + b));
+            ++gsm;
+            continue;
+          }
+          // the first block this row selects sets the reference
+          const bool first = C::PAIR ? (m == -INFINITY) : (i == 0);
           const int klen = block_len(g, j);
           uint32_t sr[CPW];
 #pragma unroll
@@ -592,7 +699,7 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           // while the exchange completes; the rare block that does exceed it
           // rescales O and goes round once more with the new reference.
           float ref = m;
-          if (i == 0) {
+          if (first) {
             ok = wwait(C::B_X + b, ph);
             if (!ok) break;
             float mx = xm[t];
@@ -634,13 +741,12 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
                 const float2 pp = ((e & 7) == 5) ? exp2_poly2(x)
                                                  : make_float2(ex2_approx(x.x), ex2_approx(x.y));
                 pk[e] = pack_bf16x2(pp.x, pp.y);
-                // row sum of the bf16 values the P.V product uses, so that each
-                // output row is an exact convex combination of V rows
-                acc[e & 3] = fadd2(acc[e & 3], make_float2(__uint_as_float(pk[e] << 16),
-                                                           __uint_as_float(pk[e] & 0xFFFF0000u)));
+                // row sum of the fp32 values (the bf16 rounding of P moves a
+                // row's normalisation by ~2^-9 / sqrt(keys) relative)
+                acc[e & 3] = fadd2(acc[e & 3], pp);
               }
             }
-            if (i == 0 || pass == 1) break;
+            if (first || pass == 1) break;
             ok = wwait(C::B_X + b, ph);
             if (!ok) break;
             float mx = xm[t];
@@ -723,8 +829,9 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < DPW; ++c) orr[c] = __float_as_uint(sig * __uint_as_float(orr[c]));
         }
-        if (t < BS) {
-          const float inv = qvalid ? 1.0f / lt : 0.f;
+        if (has_rows) {
+          // (a pair's row that selects no block has lt = 0: O = 0, lse = -inf)
+          const float inv = (qvalid && lt > 0.f) ? 1.0f / lt : 0.f;
 #pragma unroll
           for (int c = 0; c < DPW; c += 8) {
             uint4 v;
@@ -736,13 +843,20 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           }
           // the low-bit codes carry a factor 2^6 (the reference maps to code 104)
           const float mref = LB ? m - 6.0f : m;
-          if (P.lse && wg == 0) P.lse[orow] = qvalid ? (mref * 0.69314718055994531f + logf(lt)) : 0.f;
+          if (P.lse && wg == 0)
+            P.lse[orow] = qvalid ? (lt > 0.f ? mref * 0.69314718055994531f + logf(lt) : -INFINITY) : 0.f;
         }
       }
       if (P.trace && threadIdx.x == 0) {
-        P.trace[static_cast<int64_t>(row) * 3 + 0] = t_start;
-        P.trace[static_cast<int64_t>(row) * 3 + 1] = globaltimer_ns();
-        P.trace[static_cast<int64_t>(row) * 3 + 2] = smid();
+        // the mask row (rows, for a pair) this item covered
+        const int r0 = C::PAIR ? static_cast<int>(bh) * g.nb + static_cast<int>(iq) : row;
+        const int nr = C::PAIR && static_cast<int>(iq) + 1 < g.nb ? 2 : 1;
+        const uint64_t t_end = globaltimer_ns();
+        for (int k = 0; k < nr; ++k) {
+          P.trace[static_cast<int64_t>(r0 + k) * 3 + 0] = t_start;
+          P.trace[static_cast<int64_t>(r0 + k) * 3 + 1] = t_end;
+          P.trace[static_cast<int64_t>(r0 + k) * 3 + 2] = smid();
+        }
       }
     }
   }
@@ -861,6 +975,17 @@ __global__ void timeout_probe_kernel(Ctrl* ctrl, uint64_t budget_ns) {
   if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, budget_ns, &abort_flag, &ctrl->status);
 }
 
+// y = exp2_poly2(x) element-wise (the softmax's FMA-pipe exponential), for
+// checking it against the exact 2^x.
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 r = exp2_poly2(v);
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
+}
+
 // ----------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -969,7 +1094,8 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
   ap.lse = lse;
   ap.trace = trace;
   ap.ctrl = ctrl;
-  ap.R = p->info.rows;
+  // block size 64 (bf16): work items are pairs of query blocks
+  ap.R = (g.bs == 64 && p->g.dtype == SBA_BF16) ? g.B * g.H * ((g.nb + 1) / 2) : p->info.rows;
   ap.sched = sched;
   ap.max_nnz = p->info.max_nnz;
   ap.budget_ns = p->wait_budget_ns;
@@ -1006,6 +1132,13 @@ cudaError_t launch_attention_lowbit(const sba_plan* p, const void* qt, const voi
   ap.vexp = vexp;
   if (g.d == 128 && g.bs == 128) return launch_tc<128, 128, true>(p, qt, kt, vq, ap, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t st) {
+  const int64_t pairs = (n + 1) / 2;
+  const int threads = 256;
+  exp2_poly_kernel<<<static_cast<unsigned>((pairs + threads - 1) / threads), threads, 0, st>>>(x, y, n);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_timeout_probe(void* workspace, uint64_t timeout_ns, cudaStream_t st) {

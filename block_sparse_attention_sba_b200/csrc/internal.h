@@ -15,7 +15,9 @@ struct sba_plan {
   int esize;               // bytes per element (2 or 4)
   size_t ws_ctrl;          // offset of the control block (status, counters)
   size_t ws_qbar, ws_kbar; // offsets of the pooled means (fp64 [B*H][nb][d])
+  size_t ws_scores, scores_bytes;  // pooled scores of a chunk of heads (fp64 [heads][nb][nb])
   size_t ws_perm;          // Hilbert order: offset of token_of_slot (int32 [Npad])
+  size_t ws_heads;         // per-(b, h) counters of sba_smooth_v (uint32 [B*H], zero between calls)
   uint64_t wait_budget_ns; // bounded-wait limit for device waits
   std::vector<int32_t> slot_of_token;  // Hilbert order: int32 [N]
   std::vector<int32_t> token_of_slot;  // Hilbert order: int32 [Npad], -1 = padding
@@ -28,7 +30,10 @@ struct Ctrl {
   uint32_t status;        // kStatusTimeout | kStatusCheck bits
   uint32_t work_next;     // persistent scheduler: next work_order index
   uint32_t cta_done;      // persistent scheduler: CTAs that finished
-  uint32_t pad[61];
+  uint32_t aux_next;      // sba_smooth_v: next work item
+  uint32_t aux_done;      // sba_smooth_v: CTAs that finished
+  uint32_t scan_done;     // mask: head-scan CTAs that finished
+  uint32_t pad[58];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 
@@ -99,7 +104,8 @@ cudaError_t launch_reorder(const sba_plan* p, int direction, const void* src[3],
 cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
                               const float* top_p, int top_k, uint32_t* bitmask, int32_t* row_cnt,
                               int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
-                              double* qbar, double* kbar, uint32_t* status, cudaStream_t st);
+                              double* qbar, double* kbar, double* scores, size_t scores_bytes,
+                              Ctrl* ctrl, cudaStream_t st);
 cudaError_t launch_build_stripe_mask(const sba_plan* p, const sba_stripe* params,
                                      uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
                                      int32_t* col_idx, int32_t* work_order, void* workspace,
@@ -109,6 +115,7 @@ cudaError_t launch_attention(const sba_plan* p, const void* qt, const void* kt, 
                              const int32_t* work_order, void* ot, float* lse, int sched,
                              uint64_t* trace, void* workspace, cudaStream_t st);
 cudaError_t launch_timeout_probe(void* workspace, uint64_t timeout_ns, cudaStream_t st);
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t st);
 
 cudaError_t launch_smooth_v(const sba_plan* p, const void* vt, void* vq, float* vmean,
                             int32_t* vexp, void* workspace, cudaStream_t st);

@@ -10,9 +10,19 @@
 // E4M3(R * 2^-e) with round-to-nearest-even and saturation. The codes of a
 // block are stored transposed, [d][bs] bytes, so that a block is a K-major
 // operand of the fp8 tensor-core product (rows = channels, keys contiguous).
-// Two launches: per-block means and residual maxima, then per-block
-// quantisation (each CTA reduces its head's maxima to e).
+//
+// One persistent launch. Work items are per block: a statistics item (mu_j
+// and the block's max |R|) and a quantisation item (needs the head's e, i.e.
+// every statistics item of the head). Items are taken from a counter in the
+// order S0, S1, Q0, S2, Q1, ..., S(BH-1), Q(BH-2), Q(BH-1) (S: statistics of
+// a head's blocks, Q: its quantisation), so a quantisation item only waits on
+// items that resident CTAs have already taken (bounded wait on the head's
+// completed-statistics count), and it re-reads its block about two heads
+// after the statistics pass read it, from L2. Both item kinds stage the block
+// in shared memory with 16-byte loads. The last CTA resets the counters.
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -21,48 +31,7 @@ namespace sba {
 
 namespace {
 
-constexpr int kSmoothThreads = 128;  // one thread per channel (d <= 128)
-
-// Real-token test of slot o of block j (cube or Hilbert order): the real
-// tokens are the block's first block_len slots.
-__device__ __forceinline__ bool slot_real(const KGeom& g, int j, int o) { return o < block_len(g, j); }
-
-// grid (nb, B*H): mu_j (fp32) and max |V - mu_j| over the block's real slots.
-__global__ void __launch_bounds__(kSmoothThreads)
-    smooth_stats_kernel(KGeom g, const __nv_bfloat16* __restrict__ vt, float* __restrict__ vmean,
-                        float* __restrict__ block_amax) {
-  const int j = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-  const int64_t base = (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * g.d;
-  __shared__ float red[kSmoothThreads / 32];
-  float mu = 0.f;
-  if (c < g.d) {
-    double sum = 0.0;
-    int cnt = 0;
-    for (int o = 0; o < g.bs; ++o) {
-      if (!slot_real(g, j, o)) continue;
-      sum += static_cast<double>(__bfloat162float(vt[base + static_cast<int64_t>(o) * g.d + c]));
-      ++cnt;
-    }
-    mu = static_cast<float>(sum / static_cast<double>(cnt));
-    vmean[(static_cast<int64_t>(bh) * g.nb + j) * g.d + c] = mu;
-  }
-  float amax = 0.f;
-  if (c < g.d) {
-    for (int o = 0; o < g.bs; ++o) {
-      if (!slot_real(g, j, o)) continue;
-      const float r = __bfloat162float(vt[base + static_cast<int64_t>(o) * g.d + c]) - mu;
-      amax = fmaxf(amax, fabsf(r));
-    }
-  }
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  if ((c & 31) == 0) red[c >> 5] = amax;
-  __syncthreads();
-  if (c == 0) {
-    float m = red[0];
-    for (int w = 1; w < kSmoothThreads / 32; ++w) m = fmaxf(m, red[w]);
-    block_amax[static_cast<int64_t>(bh) * g.nb + j] = m;
-  }
-}
+constexpr int kSmoothThreads = 256;
 
 // Smallest e with amax <= 448 * 2^e (0 for amax == 0), exact in fp32.
 __device__ __forceinline__ int scale_exponent(float amax) {
@@ -81,43 +50,156 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
-// grid (nb, B*H): codes of block j, transposed to [d][bs].
-__global__ void __launch_bounds__(kSmoothThreads)
-    smooth_quant_kernel(KGeom g, const __nv_bfloat16* __restrict__ vt,
-                        const float* __restrict__ vmean, const float* __restrict__ block_amax,
-                        uint8_t* __restrict__ vq, int32_t* __restrict__ vexp) {
-  const int j = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-  __shared__ float red[kSmoothThreads / 32];
-  float amax = 0.f;
-  for (int k = c; k < g.nb; k += kSmoothThreads)
-    amax = fmaxf(amax, block_amax[static_cast<int64_t>(bh) * g.nb + k]);
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  if ((c & 31) == 0) red[c >> 5] = amax;
+struct SmoothArgs {
+  const __nv_bfloat16* vt;
+  uint8_t* vq;
+  float* vmean;
+  int32_t* vexp;
+  float* block_amax;    // [B*H][nb]
+  uint32_t* heads;      // [B*H] statistics items completed (zero between calls)
+  Ctrl* ctrl;
+  uint64_t budget_ns;
+};
+
+__device__ __forceinline__ float block_max_f(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   __syncthreads();
-  amax = red[0];
-  for (int w = 1; w < kSmoothThreads / 32; ++w) amax = fmaxf(amax, red[w]);
-  const int e = scale_exponent(amax);
-  if (j == 0 && c == 0) vexp[bh] = e;
-  if (c >= g.d) return;
-  const float inv = ldexpf(1.0f, -e);  // exact power of two
-  const float mu = vmean[(static_cast<int64_t>(bh) * g.nb + j) * g.d + c];
-  const int64_t src = (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * g.d + c;
-  uint8_t* dst = vq + ((static_cast<int64_t>(bh) * g.nb + j) * g.d + c) * g.bs;
-  for (int k0 = 0; k0 < g.bs; k0 += 16) {
-    uint32_t w[4];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = red[0];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float x[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int o = k0 + 4 * q + u;
-        x[u] = slot_real(g, j, o)
-                   ? (__bfloat162float(vt[src + static_cast<int64_t>(o) * g.d]) - mu) * inv
-                   : 0.f;
-      }
-      w[q] = e4m3x2(x[0], x[1]) | (e4m3x2(x[2], x[3]) << 16);
+  for (int w = 1; w < kSmoothThreads / 32; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+__global__ void __launch_bounds__(kSmoothThreads)
+    smooth_v_kernel(KGeom g, SmoothArgs a) {
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  __nv_bfloat16* blk = reinterpret_cast<__nv_bfloat16*>(sm_raw);  // [bs][d]
+  __shared__ double dsum[kSmoothThreads];
+  __shared__ float red[kSmoothThreads / 32];
+  __shared__ float smu[128];
+  __shared__ int s_item;
+  const int tid = threadIdx.x, d = g.d, nb = g.nb;
+  const int BH = g.B * g.H;
+  const int vpr = d / 8;  // 16-byte vectors per row
+  const uint32_t n_items = 2u * static_cast<uint32_t>(BH) * static_cast<uint32_t>(nb);
+  uint32_t* status = &a.ctrl->status;
+  for (;;) {
+    if (tid == 0) s_item = static_cast<int>(atomicAdd(&a.ctrl->aux_next, 1u));
+    __syncthreads();
+    const uint32_t item = static_cast<uint32_t>(s_item);
+    __syncthreads();
+    if (item >= n_items) break;
+    const uint32_t seg = item / static_cast<uint32_t>(nb);
+    const int j = static_cast<int>(item - seg * static_cast<uint32_t>(nb));
+    bool quant;
+    int bh;
+    if (seg == 0) {
+      quant = false;
+      bh = 0;
+    } else if (seg & 1u) {
+      bh = static_cast<int>((seg + 1) / 2);
+      quant = bh >= BH;
+      if (quant) bh = BH - 1;
+    } else {
+      quant = true;
+      bh = static_cast<int>(seg / 2) - 1;
     }
-    *reinterpret_cast<uint4*>(dst + k0) = make_uint4(w[0], w[1], w[2], w[3]);
+    const int len = block_len(g, j);
+    const __nv_bfloat16* src = a.vt + (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * d;
+    if (quant) {
+      // wait until every statistics item of the head is done
+      if (tid == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        volatile uint32_t* cnt = a.heads + bh;
+        while (*cnt < static_cast<uint32_t>(nb)) {
+          if (globaltimer_ns() - t0 > a.budget_ns) {
+            atomicOr(status, kStatusTimeout);
+            break;
+          }
+          __nanosleep(256);
+        }
+        __threadfence();
+      }
+      __syncthreads();
+    }
+    // stage the block's real rows (16-byte loads)
+    for (int v = tid; v < len * vpr; v += kSmoothThreads)
+      reinterpret_cast<uint4*>(blk)[v] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+    __syncthreads();
+    if (!quant) {
+      // per-channel sums in fp64 over the real rows: thread = (row group, channel)
+      const int groups = kSmoothThreads / d;
+      const int c = tid % d, rg = tid / d;
+      double sum = 0.0;
+      for (int o = rg; o < len; o += groups) sum += static_cast<double>(__bfloat162float(blk[o * d + c]));
+      dsum[tid] = sum;
+      __syncthreads();
+      if (tid < d) {
+        double t = 0.0;
+        for (int r = 0; r < groups; ++r) t += dsum[r * d + tid];
+        const float mu = static_cast<float>(t / static_cast<double>(len));
+        smu[tid] = mu;
+        a.vmean[(static_cast<int64_t>(bh) * nb + j) * d + tid] = mu;
+        __threadfence();  // visible device-wide before the head count moves
+      }
+      __syncthreads();
+      float amax = 0.f;
+      const float mu = smu[c];
+      for (int o = rg; o < len; o += groups)
+        amax = fmaxf(amax, fabsf(__bfloat162float(blk[o * d + c]) - mu));
+      amax = block_max_f(amax, red);
+      if (tid == 0) {
+        a.block_amax[static_cast<int64_t>(bh) * nb + j] = amax;
+        __threadfence();
+        atomicAdd(a.heads + bh, 1u);
+      }
+    } else {
+      // the head's exponent from its blocks' maxima
+      float amax = 0.f;
+      for (int k = tid; k < nb; k += kSmoothThreads)
+        amax = fmaxf(amax, __ldcg(&a.block_amax[static_cast<int64_t>(bh) * nb + k]));
+      amax = block_max_f(amax, red);
+      const int e = scale_exponent(amax);
+      if (j == 0 && tid == 0) a.vexp[bh] = e;
+      const float inv = ldexpf(1.0f, -e);  // exact power of two
+      if (tid < d) smu[tid] = __ldcg(&a.vmean[(static_cast<int64_t>(bh) * nb + j) * d + tid]);
+      __syncthreads();
+      // 16 codes of one channel per store: (channel, group of 16 slots)
+      uint8_t* dst = a.vq + (static_cast<int64_t>(bh) * nb + j) * d * g.bs;
+      const int ng = g.bs / 16;
+      for (int idx = tid; idx < d * ng; idx += kSmoothThreads) {
+        const int c = idx % d, og = idx / d;
+        const float mu = smu[c];
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int o = og * 16 + 4 * q + u;
+            x[u] = o < len ? (__bfloat162float(blk[o * d + c]) - mu) * inv : 0.f;
+          }
+          w[q] = e4m3x2(x[0], x[1]) | (e4m3x2(x[2], x[3]) << 16);
+        }
+        *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(c) * g.bs + og * 16) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    __syncthreads();
+  }
+  // the last CTA out resets the work counter and the head counters
+  if (tid == 0) {
+    __threadfence();
+    const uint32_t prev = atomicAdd(&a.ctrl->aux_done, 1u);
+    if (prev == gridDim.x - 1) {
+      for (int h = 0; h < BH; ++h) a.heads[h] = 0u;
+      atomicExch(&a.ctrl->aux_next, 0u);
+      atomicExch(&a.ctrl->aux_done, 0u);
+      __threadfence();
+    }
   }
 }
 
@@ -126,16 +208,33 @@ __global__ void __launch_bounds__(kSmoothThreads)
 cudaError_t launch_smooth_v(const sba_plan* p, const void* vt, void* vq, float* vmean,
                             int32_t* vexp, void* workspace, cudaStream_t st) {
   KGeom g = make_kgeom(p);
+  char* ws = static_cast<char*>(workspace);
+  SmoothArgs a;
+  a.vt = static_cast<const __nv_bfloat16*>(vt);
+  a.vq = static_cast<uint8_t*>(vq);
+  a.vmean = vmean;
+  a.vexp = vexp;
   // per-block residual maxima live in the pooled-means area of the workspace
-  float* block_amax = reinterpret_cast<float*>(static_cast<char*>(workspace) + p->ws_qbar);
-  dim3 grid(g.nb, g.B * g.H);
-  smooth_stats_kernel<<<grid, kSmoothThreads, 0, st>>>(g, static_cast<const __nv_bfloat16*>(vt),
-                                                       vmean, block_amax);
-  cudaError_t e = cudaGetLastError();
+  a.block_amax = reinterpret_cast<float*>(ws + p->ws_qbar);
+  a.heads = reinterpret_cast<uint32_t*>(ws + p->ws_heads);
+  a.ctrl = reinterpret_cast<Ctrl*>(ws + p->ws_ctrl);
+  a.budget_ns = p->wait_budget_ns;
+  const int smem = g.bs * g.d * 2;
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  smooth_quant_kernel<<<grid, kSmoothThreads, 0, st>>>(g, static_cast<const __nv_bfloat16*>(vt),
-                                                       vmean, block_amax,
-                                                       static_cast<uint8_t*>(vq), vexp);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(smooth_v_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smooth_v_kernel, kSmoothThreads, smem);
+  if (e != cudaSuccess) return e;
+  // persistent: every CTA resident at once (a quantisation item waits on
+  // statistics items that resident CTAs took earlier)
+  const int64_t items = 2ll * g.B * g.H * g.nb;
+  const int grid = static_cast<int>(std::min<int64_t>(items, static_cast<int64_t>(std::max(1, per_sm)) * sms));
+  smooth_v_kernel<<<grid, kSmoothThreads, smem, st>>>(g, a);
   return cudaGetLastError();
 }
 

@@ -3,19 +3,22 @@
 // "Top-p routing, a Top-k safety floor"), plus the longest-first work order
 // that absorbs the uneven per-head workloads the abstract describes.
 //
-// Four launches on the caller's stream:
+// Launches on the caller's stream:
 //   pool_kernel        mean of the real tokens of every block of qt and kt
-//                      (fp32). HBM-bound: reads qt and kt once.
-//   select_kernel      per (b, h) and 16 query blocks: pooled scores on CUDA
-//                      cores in fp32, row softmax, a warp bitonic sort of
-//                      (probability, index) keys in shared memory, a warp scan
-//                      of the sorted masses, the Top-p cut with the Top-k
-//                      floor; writes the bitmask row and row_cnt.
-//   scan_order_kernel  one CTA: row_ptr (exclusive scan of row_cnt) and the
-//                      work order (stable counting sort by row_cnt, longest
-//                      first) with per-warp segment counters, so the result is
-//                      deterministic.
-//   expand_kernel      one warp per row: bitmask -> ascending col_idx.
+//                      (summed in fp64). HBM-bound: reads qt and kt once.
+//   score_kernel       pooled scores Qbar_i . Kbar_j / sqrt(d) in fp64 for a
+//                      chunk of heads (64 x 64 tiles, fp64 FMA on CUDA cores)
+//                      into a scratch that stays in L2 until:
+//   cut_kernel         one warp per row: fp64 row softmax over the key
+//                      blocks, the Top-p cut by bisection on the probability
+//                      bits (no sort) with the Top-k floor; writes the bitmask
+//                      row and row_cnt. (score, cut) repeat per chunk of heads.
+//   head_scan_kernel   one warp per head: row_ptr within the head, the head's
+//                      longest-first order (stable counting sort, so the
+//                      result is deterministic) and total; the last CTA orders
+//                      the heads and offsets them.
+//   finalize_kernel    one warp per row: global row_ptr, the work_order entry
+//                      and the ascending col_idx from the bitmask.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -32,6 +35,17 @@ namespace {
 // ------------------------------------------------------------------ pooling
 constexpr int kPoolThreads = 256;
 
+// bf16 -> fp64 by moving the bit fields (exact): the exponent is rebiased by
+// 1023 - 127 and the 7 mantissa bits land at the top of fp64's 52. Zero,
+// subnormal, infinite and NaN inputs (exponent field 0 or 255) take the
+// conversion instructions instead.
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) {
+  const uint32_t ex = b & 0x7F80u;
+  if (ex == 0u || ex == 0x7F80u) return static_cast<double>(__uint_as_float(b << 16));
+  const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + (896u << 20));
+  return __hiloint2double(static_cast<int>(hi), 0);
+}
+
 template <typename T>
 __device__ __forceinline__ void accum_vec(double* acc, const uint4& v);
 
@@ -40,8 +54,8 @@ __device__ __forceinline__ void accum_vec<__nv_bfloat16>(double* acc, const uint
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
-    acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
+    acc[2 * i] += bf16_bits_to_f64(w[i] & 0xFFFFu);
+    acc[2 * i + 1] += bf16_bits_to_f64(w[i] >> 16);
   }
 }
 
@@ -55,9 +69,13 @@ __device__ __forceinline__ void accum_vec<float>(double* acc, const uint4& v) {
 
 // grid (nb, B*H, 2): z = 0 pools qt, z = 1 pools kt. Sums in fp64 (a sum of
 // bf16 or fp32 values is exact there for any realistic spread of exponents),
-// one division by the number of real tokens.
+// one division by the number of real tokens. Each thread issues kPoolLoads
+// 16-byte loads before it accumulates them; few registers keep four CTAs per
+// SM in flight.
+constexpr int kPoolLoads = 4;
+
 template <typename T>
-__global__ void __launch_bounds__(kPoolThreads)
+__global__ void __launch_bounds__(kPoolThreads, 4)
     pool_kernel(KGeom g, const char* __restrict__ qt, const char* __restrict__ kt,
                 double* __restrict__ qbar, double* __restrict__ kbar) {
   constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
@@ -77,9 +95,16 @@ __global__ void __launch_bounds__(kPoolThreads)
   double acc[EPV];
 #pragma unroll
   for (int e = 0; e < EPV; ++e) acc[e] = 0.0;
-  for (int o = rg; o < len; o += groups) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + o * row_bytes + c * 16));
-    accum_vec<T>(acc, v);
+  for (int o0 = rg; o0 < len; o0 += groups * kPoolLoads) {
+    uint4 v[kPoolLoads];
+#pragma unroll
+    for (int u = 0; u < kPoolLoads; ++u) {
+      const int o = o0 + u * groups;
+      if (o < len) v[u] = __ldg(reinterpret_cast<const uint4*>(base + o * row_bytes + c * 16));
+    }
+#pragma unroll
+    for (int u = 0; u < kPoolLoads; ++u)
+      if (o0 + u * groups < len) accum_vec<T>(acc, v[u]);
   }
   __shared__ double red[kPoolThreads * 8];
   // red[rg][d]: reduce over row groups
@@ -99,7 +124,6 @@ __global__ void __launch_bounds__(kPoolThreads)
 // where the cumulative mass at the cut lies within rounding of p.
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kRQ = 16;      // query blocks per CTA
 constexpr int kMaxE = 32;    // probabilities per lane (nb <= 1024)
 
 struct SelectArgs {
@@ -118,55 +142,103 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
-// grid (ceil(nb/kRQ), B*H), kSelThreads threads. Dynamic shared memory:
-//   qs [kRQ][d] f64 | S [kRQ][nb] f64
-// Phase 1: thread t computes the scores of key blocks t, t+256, ... against
-// the CTA's kRQ query blocks (fp64 FMA, K rows streamed from L1).
-// Phase 2: one warp per query block: fp64 softmax over the key blocks, then
-// the cut: the largest probability v with mass(P >= v) >= p found by
-// bisection on the bit pattern of v (warp mass sums), the ties of v taken in
-// index order until the mass reaches p; the Top-k floor by the same
-// bisection on counts. No sort.
-__global__ void __launch_bounds__(kSelThreads, 2)
-    select_kernel(KGeom g, const double* __restrict__ qbar, const double* __restrict__ kbar,
-                  SelectArgs sa, int top_k, uint32_t* __restrict__ bitmask,
-                  int32_t* __restrict__ row_cnt) {
-  extern __shared__ __align__(16) unsigned char smem[];
+// Pooled scores of a chunk of heads: S[bh - h0][i][j] = (Qbar_i . Kbar_j) / sqrt(d)
+// in fp64, each product summed over c = 0 .. d-1 in order. A CTA computes a
+// 64 x 64 tile of one head (thread: 4 x 4 outputs), with 16-column slices of
+// the two operands staged transposed in shared memory.
+// grid (ceil(nb/64), ceil(nb/64), heads in the chunk).
+constexpr int kScoreTile = 64;
+constexpr int kScoreK = 16;
+
+__global__ void __launch_bounds__(256)
+    score_kernel(KGeom g, int h0, const double* __restrict__ qbar, const double* __restrict__ kbar,
+                 double* __restrict__ S) {
+  __shared__ double qs[kScoreK][kScoreTile];
+  __shared__ double ks[kScoreK][kScoreTile];
   const int d = g.d, nb = g.nb;
-  const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * kRQ;
-  double* qs = reinterpret_cast<double*>(smem);
-  double* S = qs + kRQ * d;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = h0 + static_cast<int>(blockIdx.z);
+  const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const double* qsrc = qbar + static_cast<int64_t>(bh) * nb * d;
   const double* ksrc = kbar + static_cast<int64_t>(bh) * nb * d;
-
-  // stage the query rows (zero rows past nb)
-  for (int e = tid; e < kRQ * d; e += kSelThreads) {
-    const int r = e / d, c = e % d;
-    qs[e] = (q0 + r < nb) ? qsrc[static_cast<int64_t>(q0 + r) * d + c] : 0.0;
-  }
-  __syncthreads();
-  const double sqrt_d = sqrt(static_cast<double>(d));
-  for (int j = tid; j < nb; j += kSelThreads) {
-    double acc[kRQ];
+  double acc[4][4];
 #pragma unroll
-    for (int r = 0; r < kRQ; ++r) acc[r] = 0.0;
-    const double2* krow = reinterpret_cast<const double2*>(ksrc + static_cast<int64_t>(j) * d);
-    for (int c2 = 0; c2 < d / 2; ++c2) {
-      const double2 kv = __ldg(krow + c2);
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int r = 0; r < kRQ; ++r) {
-        const double2 qv = reinterpret_cast<const double2*>(qs + r * d)[c2];
-        acc[r] = fma(qv.x, kv.x, acc[r]);
-        acc[r] = fma(qv.y, kv.y, acc[r]);
-      }
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  // loader: thread -> (row lr, 4 columns lc..lc+3) of a 64 x 16 slice; the
+  // next slice's global loads are in flight while the current one is used
+  const int lr = tid >> 2, lc = (tid & 3) * 4;
+  const int iq = i0 + lr, jk = j0 + lr;
+  const double2* qrow = reinterpret_cast<const double2*>(qsrc + static_cast<int64_t>(min(iq, nb - 1)) * d + lc);
+  const double2* krow = reinterpret_cast<const double2*>(ksrc + static_cast<int64_t>(min(jk, nb - 1)) * d + lc);
+  const double2 z2 = make_double2(0.0, 0.0);
+  double2 q01 = iq < nb ? __ldg(qrow) : z2, q23 = iq < nb ? __ldg(qrow + 1) : z2;
+  double2 k01 = jk < nb ? __ldg(krow) : z2, k23 = jk < nb ? __ldg(krow + 1) : z2;
+  for (int c0 = 0; c0 < d; c0 += kScoreK) {
+    __syncthreads();
+    qs[lc + 0][lr] = q01.x;
+    qs[lc + 1][lr] = q01.y;
+    qs[lc + 2][lr] = q23.x;
+    qs[lc + 3][lr] = q23.y;
+    ks[lc + 0][lr] = k01.x;
+    ks[lc + 1][lr] = k01.y;
+    ks[lc + 2][lr] = k23.x;
+    ks[lc + 3][lr] = k23.y;
+    __syncthreads();
+    if (c0 + kScoreK < d) {
+      const int nx = (c0 + kScoreK) / 2;  // double2 offset of the next slice
+      q01 = iq < nb ? __ldg(qrow + nx) : z2;
+      q23 = iq < nb ? __ldg(qrow + nx + 1) : z2;
+      k01 = jk < nb ? __ldg(krow + nx) : z2;
+      k23 = jk < nb ? __ldg(krow + nx + 1) : z2;
     }
 #pragma unroll
-    for (int r = 0; r < kRQ; ++r) S[r * nb + j] = acc[r] / sqrt_d;
+    for (int c = 0; c < kScoreK; ++c) {
+      const double2 qa = *reinterpret_cast<const double2*>(&qs[c][ty * 4]);
+      const double2 qb = *reinterpret_cast<const double2*>(&qs[c][ty * 4 + 2]);
+      const double2 ka = *reinterpret_cast<const double2*>(&ks[c][tx * 4]);
+      const double2 kb = *reinterpret_cast<const double2*>(&ks[c][tx * 4 + 2]);
+      const double qv[4] = {qa.x, qa.y, qb.x, qb.y};
+      const double kv[4] = {ka.x, ka.y, kb.x, kb.y};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fma(qv[a], kv[b], acc[a][b]);
+    }
   }
-  __syncthreads();
+  const double sqrt_d = sqrt(static_cast<double>(d));
+  double* dst = S + static_cast<int64_t>(blockIdx.z) * nb * nb;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty * 4 + a;
+    if (i >= nb) continue;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + tx * 4 + b;
+      if (j < nb) dst[static_cast<int64_t>(i) * nb + j] = acc[a][b] / sqrt_d;
+    }
+  }
+}
 
+// One warp per (head, query block) row of the chunk: the row's pooled scores
+// (from score_kernel) -> fp64 softmax over the key blocks, then the cut: the
+// largest probability v with mass(P >= v) >= p found by bisection on the bit
+// pattern of v (warp mass sums), the ties of v taken in index order until the
+// mass reaches p; the Top-k floor by the same bisection on counts. No sort.
+// Writes the row's bitmask words and row_cnt. grid ceil(rows of chunk / 8).
+__global__ void __launch_bounds__(kSelThreads)
+    cut_kernel(KGeom g, int h0, int nheads, const double* __restrict__ S, SelectArgs sa, int top_k,
+               uint32_t* __restrict__ bitmask, int32_t* __restrict__ row_cnt) {
+  const int nb = g.nb;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rloc = blockIdx.x * kSelWarps + warp;  // row within the chunk
+  if (rloc >= nheads * nb) return;
+  const int bh = h0 + rloc / nb;
+  const int i = rloc % nb;
+  const double* srow = S + static_cast<int64_t>(rloc) * nb;
+  __shared__ double cbuf_all[kSelWarps][32];
+  double* cbuf = cbuf_all[warp];
   uint32_t h;
   {
     uint32_t bq;
@@ -174,21 +246,23 @@ __global__ void __launch_bounds__(kSelThreads, 2)
   }
   const double p = static_cast<double>(sa.top_p[h]);
   const int E = (nb + 31) >> 5;
-  for (int r = warp; r < kRQ; r += kSelWarps) {
-    const int i = q0 + r;
-    if (i >= nb) break;
-    const double* srow = S + r * nb;
+  {
     // softmax in fp64: shift by the row max, exp, divide by the sum
+    double pv[kMaxE];
     double mx = -INFINITY;
-    for (int j = lane; j < nb; j += 32) mx = fmax(mx, srow[j]);
+#pragma unroll
+    for (int e = 0; e < kMaxE; ++e) {
+      const int j = lane + 32 * e;
+      pv[e] = (e < E && j < nb) ? __ldcg(srow + j) : -INFINITY;
+      mx = fmax(mx, pv[e]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    double pv[kMaxE];
     double esum = 0.0;
 #pragma unroll
     for (int e = 0; e < kMaxE; ++e) {
       const int j = lane + 32 * e;
-      pv[e] = (e < E && j < nb) ? exp(srow[j] - mx) : 0.0;
+      pv[e] = (e < E && j < nb) ? exp(pv[e] - mx) : 0.0;
       esum += pv[e];
     }
     esum = warp_sum(esum);
@@ -234,12 +308,16 @@ __global__ void __launch_bounds__(kSelThreads, 2)
     // pred(mass(P >= v), count(P >= v)). Invariant: pred holds at lo and fails
     // at hi, so the answer lies in [lo, hi); stop once one element is left
     // there (or the interval is one pattern wide).
+    // Once at most 32 elements are left in [lo, hi) they are gathered one per
+    // lane (through this warp's slice of shared memory) and the remaining
+    // steps sum only them on top of the mass and count at hi.
     auto bisect = [&](bool by_mass, double p_or_n) -> unsigned long long {
       unsigned long long lo = 0ull, hi = 1ull << 62;
-      double m;
+      double m, m_hi = 0.0;
       int c_lo, c_hi = 0;
       ge_sums(0.0, m, c_lo);
-      for (int b = 61; b >= 0 && c_lo - c_hi > 1; --b) {
+      int b = 61;
+      for (; b >= 0 && c_lo - c_hi > 32; --b) {
         const unsigned long long mid = lo | (1ull << b);
         int c;
         ge_sums(as_double(mid), m, c);
@@ -250,9 +328,56 @@ __global__ void __launch_bounds__(kSelThreads, 2)
         } else {
           hi = mid;
           c_hi = c;
+          m_hi = m;
         }
       }
-      return c_lo - c_hi == 1 ? only_in(lo, hi) : lo;
+      if (c_lo - c_hi <= 1) return c_lo - c_hi == 1 ? only_in(lo, hi) : lo;
+      // gather the candidates in [lo, hi)
+      const double a = as_double(lo), bv = as_double(hi);
+      int mine = 0;
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e)
+        if (e < E && pv[e] >= a && pv[e] < bv) ++mine;
+      int incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int slot = incl - mine;
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e)
+        if (e < E && pv[e] >= a && pv[e] < bv) cbuf[slot++] = pv[e];
+      __syncwarp();
+      const double cand = lane < c_lo - c_hi ? cbuf[lane] : -1.0;
+      __syncwarp();
+      for (; b >= 0 && c_lo - c_hi > 1; --b) {
+        const unsigned long long mid = lo | (1ull << b);
+        const double vm = as_double(mid);
+        // only the candidates still in [mid, hi): those at or above hi are in
+        // the mass and count at hi already
+        const bool in = cand >= vm && cand < as_double(hi);
+        const int c = c_hi + __popc(__ballot_sync(0xffffffffu, in));
+        m = m_hi + warp_sum(in ? cand : 0.0);
+        const bool ok = by_mass ? (m >= p_or_n) : (static_cast<double>(c) >= p_or_n);
+        if (ok) {
+          lo = mid;
+          c_lo = c;
+        } else {
+          hi = mid;
+          c_hi = c;
+          m_hi = m;
+        }
+      }
+      if (c_lo - c_hi == 1) {
+        const double lo_v = as_double(lo), hi_v = as_double(hi);
+        double f = (cand >= lo_v && cand < hi_v) ? cand : -1.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) f = fmax(f, __shfl_xor_sync(0xffffffffu, f, o));
+        return static_cast<unsigned long long>(__double_as_longlong(f));
+      }
+      return lo;
     };
     // Top-p: n_p = the length of the shortest prefix, in descending order
     // (ties: lower index first), whose cumulative mass reaches p; all blocks
@@ -346,108 +471,62 @@ __global__ void __launch_bounds__(kSelThreads, 2)
 }
 
 // --------------------------------------------------- row_ptr + work order
-constexpr int kScanThreads = 1024;
-constexpr int kScanWarps = kScanThreads / 32;
+// Two launches, parallel over heads:
+//   head_scan_kernel   one warp per head: the head's total, the exclusive
+//                      scan of its rows' counts (row_ptr relative to the
+//                      head's first row, written into row_ptr) and each
+//                      row's place in the head's longest-first order (a
+//                      stable counting sort by count, descending, through a
+//                      per-warp bin table). The last CTA to finish turns the
+//                      head totals into head offsets and head ranks (heads by
+//                      total descending, ties: lower head first) and writes
+//                      row_ptr[R].
+//   finalize_kernel    one warp per row: row_ptr += the head's offset, the
+//                      row's work_order entry, and its col_idx from the
+//                      bitmask (one coalesced store per bitmask word).
+// Scratch (int32): pos [R], then head totals, offsets and ranks [3][BH].
+constexpr int kScanWarps = 8;
 
-// Exclusive scan of one value per thread across the CTA; returns the prefix
-// and writes the total to *total (shared).
-__device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+__global__ void __launch_bounds__(kScanWarps * 32)
+    head_scan_kernel(int BH, int nb, const int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_ptr,
+                     int32_t* __restrict__ scratch, Ctrl* __restrict__ ctrl) {
+  extern __shared__ int bins[];  // [kScanWarps][nb + 1]
+  __shared__ int last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int s = warp_sums[lane];
-    int si = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, si, o);
-      if (lane >= o) si += t;
-    }
-    warp_sums[lane] = si - s;
-    if (lane == 31) *total = si;
-  }
-  __syncthreads();
-  const int res = warp_sums[warp] + incl - v;
-  __syncthreads();
-  return res;
-}
-
-// One CTA of 1024 threads. Dynamic shared memory: hist [kScanWarps][nb+1]
-// ints (one bin table per warp), head totals [BH] and head ranks [BH].
-// Work order: heads by total selected blocks descending (ties: lower head
-// first), then, inside a head, rows by count descending (ties: lower row
-// first). Each warp sorts whole heads with a stable counting sort over its own
-// bin table, so the result is deterministic.
-__global__ void __launch_bounds__(kScanThreads)
-    scan_order_kernel(int R, int nb, int BH, const int32_t* __restrict__ row_cnt,
-                      int32_t* __restrict__ row_ptr, int32_t* __restrict__ work_order,
-                      uint32_t* __restrict__ status) {
-  extern __shared__ int ssm[];
-  __shared__ int warp_sums[32];
-  __shared__ int total;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nc = nb + 1;
-  int* hist = ssm;                         // [kScanWarps][nc]
-  int* htot = hist + kScanWarps * nc;      // [BH]
-  int* hrank = htot + BH;                  // [BH]
-
-  // ---- row_ptr: each thread owns a contiguous chunk of rows
-  const int per = (R + kScanThreads - 1) / kScanThreads;
-  const int r0 = min(R, tid * per), r1 = min(R, r0 + per);
-  int local = 0;
-  for (int r = r0; r < r1; ++r) local += row_cnt[r];
-  int run = block_exclusive_scan(local, warp_sums, &total);
-  for (int r = r0; r < r1; ++r) {
-    row_ptr[r] = run;
-    run += row_cnt[r];
-  }
-  if (tid == 0) row_ptr[R] = total;
-
-  // ---- head totals (one warp per head)
-  for (int h = warp; h < BH; h += kScanWarps) {
-    int sum = 0;
-    for (int i = lane; i < nb; i += 32) sum += row_cnt[h * nb + i];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) htot[h] = sum;
-  }
-  __syncthreads();
-  // ---- head ranks: number of heads that come first
-  for (int h = tid; h < BH; h += kScanThreads) {
-    const int th = htot[h];
-    int rk = 0;
-    for (int x = 0; x < BH; ++x) {
-      const int tx = htot[x];
-      rk += (tx > th) || (tx == th && x < h);
-    }
-    hrank[h] = rk;
-  }
-  __syncthreads();
-
-  // ---- inside each head: stable counting sort by count, descending
-  int* myh = hist + warp * nc;
-  for (int h = warp; h < BH; h += kScanWarps) {
+  const int R = BH * nb, nc = nb + 1;
+  int32_t* pos = scratch;
+  int32_t* htot = scratch + R;
+  int32_t* hoff = htot + BH;
+  int32_t* hrank = hoff + BH;
+  const int h = blockIdx.x * kScanWarps + warp;
+  if (h < BH) {
+    int* myh = bins + warp * nc;
     for (int c = lane; c < nc; c += 32) myh[c] = 0;
     __syncwarp();
     const int base_row = h * nb;
+    // counts, the within-head exclusive scan, and the histogram of counts
+    int run = 0;
     for (int b = 0; b < nb; b += 32) {
       const int i = b + lane;
       const bool act = i < nb;
-      int c = act ? row_cnt[base_row + i] : -1;
+      int c = act ? row_cnt[base_row + i] : 0;
       if (act && (c < 0 || c > nb)) {
-        atomicOr(status, kStatusCheck);
+        atomicOr(&ctrl->status, kStatusCheck);
         c = 0;
       }
-      const unsigned m = __match_any_sync(0xffffffffu, c);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      if (act) row_ptr[base_row + i] = run + incl - c;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+      const unsigned m = __match_any_sync(0xffffffffu, act ? c : -1);
       if (act && lane == __ffs(m) - 1) myh[c] += __popc(m);
       __syncwarp();
     }
+    if (lane == 0) htot[h] = run;
     // start of each count's run = rows with a larger count: scan bins from nb down
     const int seg = (nc + 31) / 32;
     const int q0 = min(nc, lane * seg), q1 = min(nc, q0 + seg);
@@ -467,7 +546,6 @@ __global__ void __launch_bounds__(kScanThreads)
       rs += t;
     }
     __syncwarp();
-    const int out_base = hrank[h] * nb;
     for (int b = 0; b < nb; b += 32) {
       const int i = b + lane;
       const bool act = i < nb;
@@ -475,24 +553,67 @@ __global__ void __launch_bounds__(kScanThreads)
       if (act && (c < 0 || c > nb)) c = 0;
       const unsigned m = __match_any_sync(0xffffffffu, c);
       const int rank = __popc(m & ((1u << lane) - 1u));
-      const int pos = act ? myh[c] + rank : 0;
+      if (act) pos[base_row + i] = myh[c] + rank;
       __syncwarp();
-      if (act) work_order[out_base + pos] = base_row + i;
       if (act && lane == __ffs(m) - 1) myh[c] += __popc(m);
       __syncwarp();
     }
   }
+  // the last CTA out: head offsets (exclusive scan of the totals) and ranks
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&ctrl->scan_done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (warp == 0) {
+    int run = 0;
+    for (int b = 0; b < BH; b += 32) {
+      const int x = b + lane;
+      const int t = x < BH ? __ldcg(&htot[x]) : 0;
+      int incl = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (x < BH) hoff[x] = run + incl - t;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) row_ptr[R] = run;
+  }
+  for (int x = threadIdx.x; x < BH; x += blockDim.x) {
+    const int tx = __ldcg(&htot[x]);
+    int rk = 0;
+    for (int y = 0; y < BH; ++y) {
+      const int ty = __ldcg(&htot[y]);
+      rk += (ty > tx) || (ty == tx && y < x);
+    }
+    hrank[x] = rk;
+  }
+  if (threadIdx.x == 0) ctrl->scan_done = 0u;
 }
 
-// ------------------------------------------------------------- CSR expand
 __global__ void __launch_bounds__(256)
-    expand_kernel(int R, int nb, const uint32_t* __restrict__ bitmask,
-                  const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx) {
+    finalize_kernel(int BH, int nb, const uint32_t* __restrict__ bitmask, const int32_t* __restrict__ scratch,
+                    int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+                    int32_t* __restrict__ work_order) {
   const int lane = threadIdx.x & 31;
+  const int R = BH * nb;
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= R) return;
+  const int h = r / nb;
+  const int32_t* pos = scratch;
+  const int32_t* hoff = scratch + R + BH;
+  const int32_t* hrank = hoff + BH;
+  const int start = row_ptr[r] + hoff[h];
+  if (lane == 0) {
+    row_ptr[r] = start;
+    work_order[hrank[h] * nb + pos[r]] = r;
+  }
+  // col_idx: bit `lane` of word e lands after the set bits below it
   const int nwords = (nb + 31) >> 5;
-  uint32_t w = lane < nwords ? bitmask[static_cast<int64_t>(r) * nwords + lane] : 0u;
+  const uint32_t w = lane < nwords ? bitmask[static_cast<int64_t>(r) * nwords + lane] : 0u;
   const int cnt = __popc(w);
   int incl = cnt;
 #pragma unroll
@@ -500,46 +621,44 @@ __global__ void __launch_bounds__(256)
     const int t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
   }
-  int pos = row_ptr[r] + incl - cnt;
-  while (w) {
-    const int b = __ffs(w) - 1;
-    col_idx[pos++] = lane * 32 + b;
-    w &= w - 1;
+  const int excl = incl - cnt;
+  for (int e = 0; e < nwords; ++e) {
+    const uint32_t we = __shfl_sync(0xffffffffu, w, e);
+    const int pe = __shfl_sync(0xffffffffu, excl, e);
+    if ((we >> lane) & 1u) col_idx[start + pe + __popc(we & ((1u << lane) - 1u))] = e * 32 + lane;
   }
 }
 
 // row_ptr (exclusive scan of row_cnt), work_order and col_idx from bitmask
-// and row_cnt: shared by the Top-p and the stripe masks.
+// and row_cnt: shared by the Top-p and the stripe masks. iscratch: int32
+// [R + 3*B*H] of workspace the caller no longer needs.
 cudaError_t launch_scan_expand(const sba_plan* p, const uint32_t* bitmask, const int32_t* row_cnt,
                                int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
-                               uint32_t* status, cudaStream_t st) {
+                               int32_t* iscratch, Ctrl* ctrl, cudaStream_t st) {
   const int R = p->info.rows;
   const int nb = p->info.nb;
   const int BH = p->g.B * p->g.H;
-  const size_t scan_smem = (static_cast<size_t>(kScanWarps) * (nb + 1) + 2 * static_cast<size_t>(BH)) * sizeof(int);
-  if (scan_smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(scan_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(scan_smem));
+  const size_t smem = static_cast<size_t>(kScanWarps) * (nb + 1) * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(head_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  scan_order_kernel<<<1, kScanThreads, scan_smem, st>>>(R, nb, BH, row_cnt, row_ptr, work_order,
-                                                        status);
+  head_scan_kernel<<<(BH + kScanWarps - 1) / kScanWarps, kScanWarps * 32, smem, st>>>(
+      BH, nb, row_cnt, row_ptr, iscratch, ctrl);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  expand_kernel<<<(R + 7) / 8, 256, 0, st>>>(R, nb, bitmask, row_ptr, col_idx);
+  finalize_kernel<<<(R + 7) / 8, 256, 0, st>>>(BH, nb, bitmask, iscratch, row_ptr, col_idx, work_order);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-static size_t select_smem_bytes(int d, int nb) {
-  return static_cast<size_t>(kRQ) * d * sizeof(double) + static_cast<size_t>(kRQ) * nb * sizeof(double);
-}
-
 cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
                               const float* top_p, int top_k, uint32_t* bitmask, int32_t* row_cnt,
                               int32_t* row_ptr, int32_t* col_idx, int32_t* work_order,
-                              double* qbar, double* kbar, uint32_t* status, cudaStream_t st) {
+                              double* qbar, double* kbar, double* scores, size_t scores_bytes,
+                              Ctrl* ctrl, cudaStream_t st) {
   KGeom g = make_kgeom(p);
   const int BH = g.B * g.H;
 
@@ -553,20 +672,26 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const size_t sel_smem = select_smem_bytes(g.d, g.nb);
-  if (sel_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sel_smem));
-    if (e != cudaSuccess) return e;
-  }
   SelectArgs sa;
   for (int h = 0; h < 256; ++h) sa.top_p[h] = h < g.H ? top_p[h] : 1.0f;
-  dim3 sg((g.nb + kRQ - 1) / kRQ, BH);
-  select_kernel<<<sg, kSelThreads, sel_smem, st>>>(g, qbar, kbar, sa, top_k, bitmask, row_cnt);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  // scores then cut, a chunk of heads at a time (the chunk's scores fit the
+  // scratch and stay in L2 between the two launches)
+  const size_t per_head = static_cast<size_t>(g.nb) * g.nb * sizeof(double);
+  const int hc = static_cast<int>(std::min<size_t>(BH, scores_bytes / per_head));
+  if (hc < 1) return cudaErrorInvalidValue;
+  const int nt = (g.nb + kScoreTile - 1) / kScoreTile;
+  for (int h0 = 0; h0 < BH; h0 += hc) {
+    const int nh = std::min(hc, BH - h0);
+    score_kernel<<<dim3(nt, nt, nh), 256, 0, st>>>(g, h0, qbar, kbar, scores);
+    cut_kernel<<<(nh * g.nb + kSelWarps - 1) / kSelWarps, kSelThreads, 0, st>>>(
+        g, h0, nh, scores, sa, top_k, bitmask, row_cnt);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
 
-  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order, status, st);
+  // the pooled query means are no longer needed: their space is the scan's scratch
+  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order,
+                            reinterpret_cast<int32_t*>(qbar), ctrl, st);
 }
 
 // ------------------------------------------------------------ stripe masks
@@ -638,7 +763,8 @@ cudaError_t launch_build_stripe_mask(const sba_plan* p, const sba_stripe* params
   stripe_kernel<<<grid, 256, 0, st>>>(g, sa, bitmask, row_cnt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order, &ctrl->status, st);
+  return launch_scan_expand(p, bitmask, row_cnt, row_ptr, col_idx, work_order,
+                            reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + p->ws_qbar), ctrl, st);
 }
 
 // ------------------------------------------------------------------------
@@ -696,7 +822,11 @@ size_t noalloc_pooled_bytes(const sba_plan* p) {
   return (static_cast<size_t>(p->info.rows) * p->g.d * sizeof(double) + 255) & ~size_t(255);
 }
 
-size_t noalloc_scratch_need(const sba_plan* p) { return sizeof(Ctrl) + 2 * noalloc_pooled_bytes(p); }
+// control block, pooled means, then at least one head's pooled scores
+size_t noalloc_scratch_need(const sba_plan* p) {
+  return sizeof(Ctrl) + 2 * noalloc_pooled_bytes(p) +
+         static_cast<size_t>(p->info.nb) * p->info.nb * sizeof(double);
+}
 
 }  // namespace
 
@@ -729,7 +859,7 @@ extern "C" sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* q
   }
   const size_t need = noalloc_scratch_need(plan);
   if (need > kNoAllocScratchBytes) {
-    set_error("sba_build_mask_noalloc needs %zu bytes of scratch (2*B*H*nb*d doubles + 256) but "
+    set_error("sba_build_mask_noalloc needs %zu bytes of scratch (2*B*H*nb*d + nb*nb doubles + 256) but "
               "its static scratch holds %zu; use sba_build_mask with a workspace",
               need, kNoAllocScratchBytes);
     return SBA_ERR_CAPACITY;
@@ -745,11 +875,14 @@ extern "C" sba_status sba_build_mask_noalloc(const sba_plan* plan, const void* q
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(sc);
   double* qbar = reinterpret_cast<double*>(sc + sizeof(Ctrl));
   double* kbar = reinterpret_cast<double*>(sc + sizeof(Ctrl) + noalloc_pooled_bytes(plan));
+  // the rest of the scratch holds pooled scores, as many heads at a time as fit
+  const size_t scores_off = sizeof(Ctrl) + 2 * noalloc_pooled_bytes(plan);
+  double* scores = reinterpret_cast<double*>(sc + scores_off);
   // the control block keeps the previous call's contents: start from zero
   e = cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), st);
   if (e == cudaSuccess)
     e = launch_build_mask(plan, qt, kt, top_p, top_k, bitmask, row_cnt, row_ptr, col_idx, work_order,
-                          qbar, kbar, &ctrl->status, st);
+                          qbar, kbar, scores, kNoAllocScratchBytes - scores_off, ctrl, st);
   if (e != cudaSuccess) {
     set_error("sba_build_mask_noalloc launch: %s", cudaGetErrorString(e));
     return SBA_ERR_CUDA;

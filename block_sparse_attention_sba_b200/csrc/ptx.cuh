@@ -367,8 +367,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 2^x for a pair of floats on the FMA/ALU pipes (no MUFU), used to take part
 // of the softmax exponentials off the MUFU pipe. Method: round-to-nearest
 // range reduction with the 1.5*2^23 shifter (r = round(x), f = x - r in
-// [-1/2, 1/2]), 2^f from a degree-3 polynomial fitted here by weighted least
-// squares on Chebyshev nodes (max relative error 7.5e-5 in fp32, far below the
+// [-1/2, 1/2]), 2^f from the degree-3 polynomial of least maximum relative
+// error on that interval (Remez exchange; fit_exp2_poly.py beside this file
+// prints the coefficients: max relative error 7.5e-5 in fp32, far below the
 // bf16 rounding of P), and r added to the exponent field. x is clamped to
 // >= -125 so the result stays a normal float (2^-125 ~ 0 for P).
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
@@ -378,7 +379,7 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 j = fadd2(x, make_float2(kShift, kShift));
   const float2 r = fadd2(j, make_float2(-kShift, -kShift));
   const float2 f = fadd2(x, make_float2(-r.x, -r.y));
-  float2 p = ffma2(make_float2(0.055171605f, 0.055171605f), f, make_float2(0.24261111f, 0.24261111f));
+  float2 p = ffma2(make_float2(0.055171669f, 0.055171669f), f, make_float2(0.24261113f, 0.24261113f));
   p = ffma2(p, f, make_float2(0.69326097f, 0.69326097f));
   p = ffma2(p, f, make_float2(0.99992806f, 0.99992806f));
   return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),

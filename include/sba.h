@@ -179,8 +179,9 @@ SBA_API sba_status sba_unreorder(const sba_plan* plan, const void* ot, void* o,
  * are fp64 (the cut is found by bisection on the probabilities, not by a
  * sort), so a row can differ from another fp64 evaluation only where its
  * cumulative mass at the cut lies within rounding (~1e-15) of p.
- * The workspace holds the pooled means (2*B*H*nb*d doubles) and the status
- * word that device-side checks set. */
+ * The workspace holds the pooled means (2*B*H*nb*d doubles), the pooled
+ * scores of a chunk of heads (nb*nb doubles per head; as many heads as 48 MiB
+ * hold, at least one) and the status word that device-side checks set. */
 SBA_API sba_status sba_build_mask(const sba_plan* plan, const void* qt, const void* kt,
                           const float* top_p, int32_t top_k,
                           uint32_t* bitmask, int32_t* row_cnt, int32_t* row_ptr,
@@ -189,20 +190,22 @@ SBA_API sba_status sba_build_mask(const sba_plan* plan, const void* qt, const vo
 
 /* Allocation-free sba_build_mask (the paper has no counterpart: this is a
  * deployment convenience). Same inputs, outputs and results as sba_build_mask,
- * but no workspace argument: its scratch (the pooled block means and a
- * 256-byte control block) lives in one 64 MiB array of static device memory
+ * but no workspace argument: its scratch (a 256-byte control block, the
+ * pooled block means and the pooled scores of as many heads as fit in the
+ * rest) lives in one 64 MiB array of static device memory
  * inside the library, which every GPU that loads libsba holds until the
  * process exits. For callers that cannot allocate device memory or carry a
  * workspace: plugin interfaces that pass only inputs and outputs, and services
  * that reserve all device memory at start-up and forbid cudaMalloc afterwards.
- * Limit: 2*B*H*nb*d*8 bytes (rounded up to 256 each) + 256 <= 64 MiB, i.e.
- * B*H*nb*d <= ~4.19 million (the Wan and HunyuanVideo-shaped layers fit);
- * larger plans return SBA_ERR_CAPACITY before anything is launched.
+ * Limit: 256 + 2*B*H*nb*d*8 bytes (the two rounded up to 256 each) + one
+ * head's nb*nb*8 bytes of scores <= 64 MiB (the Wan and HunyuanVideo-shaped
+ * layers fit); larger plans return SBA_ERR_CAPACITY before anything is
+ * launched.
  * Each call looks up the array's device address on the current device with
  * cudaGetSymbolAddress (a failed lookup is reported, not remembered); inside a
  * stream capture it reuses the last address found on that device, so make one
  * call on each device before capturing. Each call clears the control block
- * with cudaMemsetAsync and overwrites the pooled means; the array keeps the
+ * with cudaMemsetAsync and overwrites the means and scores; the array keeps the
  * last call's contents. All calls share the one array, so calls that overlap
  * on the GPU (other streams, other threads) race: serialise them. Device-side
  * check failures of the call land in the array's status word: read them with
@@ -328,6 +331,14 @@ SBA_API sba_status sba_check_device_status(const sba_plan* plan, void* workspace
  * leaving the context usable. Used to test the timeout path without a hang. */
 SBA_API sba_status sba_debug_timeout_probe(const sba_plan* plan, void* workspace,
                                    uint64_t timeout_ns, void* stream);
+
+/* Numerical probe of the attention softmax's FMA-pipe exponential: y[i] =
+ * 2^x[i] as the kernel computes it for one exponential pair in eight (range
+ * reduction to f in [-1/2, 1/2], a degree-3 minimax polynomial for 2^f,
+ * x clamped at -125). x, y: device fp32 [n], 0 <= n <= 2^31; asynchronous on
+ * `stream`. The pages have no counterpart: it exists to test that
+ * approximation against the exact 2^x. */
+SBA_API sba_status sba_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
 /* Host-only: write the slot of every raster token, int32 [N]. */
 SBA_API sba_status sba_perm_export(const sba_plan* plan, int32_t* slot_of_token);

@@ -22,7 +22,7 @@ def sba():
 def _declared_symbols():
     text = open(os.path.join(ROOT, "include", "sba.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(sba_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(sba_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():

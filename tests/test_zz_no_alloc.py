@@ -69,3 +69,29 @@ def test_noalloc_rejects_a_plan_larger_than_its_scratch():
                                    fake)
     assert e.value.status == sba.SBA_ERR_CAPACITY
     assert "scratch" in sba.sba_last_error()
+
+
+def test_a_failed_call_is_not_remembered():
+    """A call that fails (here an unaligned input, rejected before any device
+    access) leaves nothing behind: the next good call succeeds, its error
+    text is empty and its routing equals the workspace path's."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_sparse_attention_sba_b200 as sba
+    wl = datagen.custom("noalloc_c", 1, 2, 5, 20, 19, 128, (2, 8, 8), top_p=(0.85, 0.9), top_k=2,
+                        rope_split=(44, 42, 42))
+    dev = torch.device("cuda:0")
+    q, k, v = datagen.generate(wl, seed=4, device=dev)
+    plan = sba.Plan.for_tensor(q, wl.T, wl.Hh, wl.W, wl.cube)
+    sa = sba.SparseAttention(plan, device=dev)
+    with pytest.raises(sba.SbaError) as e:
+        sba.sba_build_mask_noalloc(plan.handle, sa.qt.data_ptr() + 2, sa.kt, wl.top_p_per_head(),
+                                   wl.top_k, sa.bitmask, sa.row_cnt, sa.row_ptr, sa.col_idx,
+                                   sa.work_order)
+    assert e.value.status == sba.SBA_ERR_INVALID_ARG
+    ref = _routing(sba, wl, use_noalloc=False)
+    got = _routing(sba, wl, use_noalloc=True)
+    assert sba.sba_last_error() == ""
+    for key in ref:
+        assert np.array_equal(ref[key], got[key]), key
+    assert sba.sba_noalloc_status() == sba.SBA_OK
