@@ -48,6 +48,10 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sched-report", action="store_true")
     ap.add_argument("--no-lowbit", action="store_true", help="skip the low-bit P.V measurement")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the Top-p 0.5 / 0.7 report")
+    ap.add_argument("--sched-workload", default="stress",
+                    help="workload of the scheduler report (LPT persistent vs head-major grid)")
+    ap.add_argument("--sched-reps", type=int, default=3, help="launches per schedule in that report")
     ap.add_argument("--report-all", action="store_true",
                     help="per-call timings, rooflines, density and SM idle for every workload "
                          "(one JSON line each; not the benchmark line)")
@@ -424,9 +428,14 @@ def run_ours(args):
     lens = _block_lens(wl)
     nb = plan.info.nb
     f_valid = 0.0
+    f_exec = 0.0
     for r in range(len(rc)):
         li = lens[r % nb]
-        f_valid += 4.0 * wl.d * li * sum(lens[j] for j in cols[rp[r]:rp[r + 1]])
+        sel = cols[rp[r]:rp[r + 1]]
+        f_valid += 4.0 * wl.d * li * sum(lens[j] for j in sel)
+        # the kernel runs every query slot of the tile (M = 128) against the
+        # key block's real length rounded up to 16 (N of S, K of P.V)
+        f_exec += 4.0 * wl.d * bs * sum(-(-lens[j] // 16) * 16 for j in sel)
     density = nnz / (len(rc) * nb)
 
     peak, peak_sus, hbm, peak_kind = _peaks()
@@ -438,32 +447,61 @@ def run_ours(args):
     ms_calls = {k: round(statistics.mean(vv), 4) for k, vv in per_call.items()}
     overhead = (ms_calls["reorder"] + ms_calls["build_mask"] + ms_calls["unreorder"]) / ms_calls["attention"]
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API with pinned host buffers: each step
+    # copies its q, k, v in and its output back out. Copies run on two copy
+    # streams (host->device, device->host) against the compute stream with two
+    # device buffer sets, so step s+1's inputs and step s-1's output move while
+    # step s computes.
     e2e = None
     if not args.no_e2e:
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
-        n_e2e = max(3, min(args.steps, 10))
+        bufs = [tuple(torch.empty_like(x) for x in (q, k, v, o)) for _ in range(2)]
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        n_e2e = max(4, min(args.steps, 12))
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+
+        def h2d(i):
+            b = bufs[i % 2]
+            with torch.cuda.stream(h2d_s):
+                if i >= 2:
+                    h2d_s.wait_event(ev_done[i % 2])  # step i-2 no longer reads this set
+                b[0].copy_(hq, non_blocking=True)
+                b[1].copy_(hk, non_blocking=True)
+                b[2].copy_(hv, non_blocking=True)
+                ev_in[i % 2].record(h2d_s)
+
         if pg:
             pg.barrier()
         torch.cuda.synchronize(dev)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            sa(dq, dk, dv, top_p, wl.top_k, o=o, stream=stream)
-            ho.copy_(o, non_blocking=True)
-        e1.record(stream)
+        e0.record(h2d_s)
+        h2d(0)
+        for i in range(n_e2e):
+            b = bufs[i % 2]
+            if i + 1 < n_e2e:
+                h2d(i + 1)
+            stream.wait_event(ev_in[i % 2])
+            if i >= 2:
+                stream.wait_event(ev_out[i % 2])  # step i-2's output has left this set
+            sa(b[0], b[1], b[2], top_p, wl.top_k, o=b[3], stream=stream)
+            ev_done[i % 2].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_done[i % 2])
+                ho.copy_(b[3], non_blocking=True)
+                ev_out[i % 2].record(d2h_s)
+        e1.record(d2h_s)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, pg, dev)
-        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+        h2d_bytes = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
         e2e = {"value": whole_job_tflops(f_tile, ws, e2e_ms), "unit": UNIT,
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": ho.numel() * ho.element_size()}
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d_bytes,
+               "d2h_bytes_per_step": ho.numel() * ho.element_size(),
+               "steps": n_e2e, "copies": "overlapped with compute (two copy streams, two buffer sets)",
+               "ratio_to_device_step": e2e_ms / mean_step}
 
     # the low-bit P.V path (E4M3 probabilities and values) on the same inputs:
     # informational, not the headline (reduced precision)
@@ -497,7 +535,42 @@ def run_ours(args):
 
     sched = None
     if not args.no_sched_report:
-        sched = sched_report(dev)
+        sched = sched_report(dev, args.sched_workload, args.sched_reps)
+
+    # the same layer at lower Top-p (sparser routing): per-call ms, density,
+    # overhead and attention TFLOPS (a report, not the headline)
+    sweep = None
+    if not args.no_sweep and wl.name == "wan":
+        sweep = []
+        for p_sw in (0.5, 0.7):
+            tp = [p_sw] * wl.H
+            t = {"reorder": [], "build_mask": [], "attention": [], "unreorder": []}
+            for it in range(3 + 5):
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+                flush.zero_()
+                ev[0].record(stream)
+                sba.sba_reorder(h, q, k, v, sa.qt, sa.kt, sa.vt, sa.workspace, stream)
+                ev[1].record(stream)
+                sba.sba_build_mask(h, sa.qt, sa.kt, tp, wl.top_k, sa.bitmask, sa.row_cnt, sa.row_ptr,
+                                   sa.col_idx, sa.work_order, sa.workspace, stream)
+                ev[2].record(stream)
+                sba.sba_attention(h, sa.qt, sa.kt, sa.vt, sa.row_ptr, sa.col_idx, sa.work_order, sa.ot,
+                                  sa.lse, sba.SBA_SCHED_LPT, None, sa.workspace, stream)
+                ev[3].record(stream)
+                sba.sba_unreorder(h, sa.ot, o, sa.workspace, stream)
+                ev[4].record(stream)
+                torch.cuda.synchronize(dev)
+                if it >= 3:
+                    for kk, (a0, a1) in zip(t, [(0, 1), (1, 2), (2, 3), (3, 4)]):
+                        t[kk].append(ev[a0].elapsed_time(ev[a1]))
+            nnz_sw = int(sa.row_ptr[-1].item())
+            ms_sw = {kk: round(statistics.mean(vv), 4) for kk, vv in t.items()}
+            sweep.append({"top_p": p_sw, "density": nnz_sw / (len(rc) * nb), "ms_per_call": ms_sw,
+                          "overhead_frac": (ms_sw["reorder"] + ms_sw["build_mask"] + ms_sw["unreorder"])
+                          / ms_sw["attention"],
+                          "attention_tflops_tile": 4.0 * bs * bs * wl.d * nnz_sw
+                          / (ms_sw["attention"] * 1e-3) / 1e12})
+        assert sa.check(stream) == 0
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -516,6 +589,8 @@ def run_ours(args):
             "ms_per_call": ms_calls,
             "attention": {"tflops_tile": achieved,
                           "tflops_valid": f_valid / (attn_ms * 1e-3) / 1e12,
+                          "tflops_executed": f_exec / (attn_ms * 1e-3) / 1e12,
+                          "valid_over_executed": f_valid / f_exec,
                           "frac_of_peak": achieved / peak, "peak_kind": peak_kind,
                           "frac_of_sustained_peak": achieved / peak_sus if peak_sus else None},
             "overhead_frac": overhead,
@@ -523,7 +598,7 @@ def run_ours(args):
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": f_tile},
-            "scheduler": sched, "lowbit": lowbit,
+            "scheduler": sched, "lowbit": lowbit, "sparsity_sweep": sweep,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 7 * args.steps,
             "clocks": clocks, "device_status": sba.sba_status_string(status),
         }

@@ -88,6 +88,10 @@ WORKLOADS = {
     # reordered q/k/v (still larger than L2), used for profiler captures
     "wan8": Workload("wan8", 1, 8, 21, 30, 52, 128, (2, 8, 8), "bf16", (0.9,), 8,
                      rope_split=(44, 42, 42)),
+    # the stress recipe on 10 heads (each Top-p value twice), for profiler
+    # captures of the two schedules
+    "stress10": Workload("stress10", 1, 10, 21, 30, 52, 128, (2, 8, 8), "bf16", STRESS_P, 8,
+                         rope_split=(44, 42, 42), amp_range=(0.2, 3.0)),
 }
 
 
