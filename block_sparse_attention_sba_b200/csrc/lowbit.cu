@@ -125,9 +125,21 @@ __global__ void __launch_bounds__(kSmoothThreads)
       }
       __syncthreads();
     }
-    // stage the block's real rows (16-byte loads)
-    for (int v = tid; v < len * vpr; v += kSmoothThreads)
-      reinterpret_cast<uint4*>(blk)[v] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+    // stage the block's real rows (16-byte loads, four in flight per thread)
+    const int nvec = len * vpr;
+    for (int v0 = tid; v0 < nvec; v0 += 4 * kSmoothThreads) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * kSmoothThreads;
+        if (v < nvec) r[u] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * kSmoothThreads;
+        if (v < nvec) reinterpret_cast<uint4*>(blk)[v] = r[u];
+      }
+    }
     __syncthreads();
     if (!quant) {
       // per-channel sums in fp64 over the real rows: thread = (row group, channel)
