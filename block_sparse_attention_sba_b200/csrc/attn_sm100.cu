@@ -406,7 +406,9 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           }
         }
         if (lane == 0) {
-          (isv ? klen_v : klen_k)[s] = block_len(g, j);
+          // (not for the low-bit kernel: measured, the record slowed it by
+          // 13 % and its S products run over whole blocks)
+          if constexpr (!LB) (isv ? klen_v : klen_k)[s] = block_len(g, j);
           if (LB && isv) {
             // E4M3 codes of block j, [d][bs] bytes: one 128-byte-wide box
             const uint32_t dst = smem_u32(sV + s * C::VTILE_BYTES);
@@ -474,7 +476,7 @@ __global__ void __launch_bounds__(Cfg<D, BS, LB>::THREADS, 1)
           const uint32_t k_addr = smem_u32(sK + s * C::TILE_BYTES);
           // S over the block's real keys only, rounded up to the MMA's N step
           // of 16 (the softmax masks the rest of the row)
-          const uint32_t idesc_s = idesc_bf16_f32(C::M, (klen_k[s] + 15) & ~15, 0, 0);
+          const uint32_t idesc_s = idesc_bf16_f32(C::M, LB ? BS : ((klen_k[s] + 15) & ~15), 0, 0);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk & 3) * 32;
