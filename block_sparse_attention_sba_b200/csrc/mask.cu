@@ -33,18 +33,6 @@ namespace sba {
 namespace {
 
 // ------------------------------------------------------------------ pooling
-constexpr int kPoolThreads = 256;
-
-// bf16 -> fp64 by moving the bit fields (exact): the exponent is rebiased by
-// 1023 - 127 and the 7 mantissa bits land at the top of fp64's 52. Zero,
-// subnormal, infinite and NaN inputs (exponent field 0 or 255) take the
-// conversion instructions instead.
-__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) {
-  const uint32_t ex = b & 0x7F80u;
-  if (ex == 0u || ex == 0x7F80u) return static_cast<double>(__uint_as_float(b << 16));
-  const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + (896u << 20));
-  return __hiloint2double(static_cast<int>(hi), 0);
-}
 
 template <typename T>
 __device__ __forceinline__ void accum_vec(double* acc, const uint4& v);
@@ -54,8 +42,9 @@ __device__ __forceinline__ void accum_vec<__nv_bfloat16>(double* acc, const uint
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += bf16_bits_to_f64(w[i] & 0xFFFFu);
-    acc[2 * i + 1] += bf16_bits_to_f64(w[i] >> 16);
+    // bf16 -> fp32 is a shift (exact), fp32 -> fp64 exact
+    acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
+    acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
   }
 }
 
@@ -67,55 +56,60 @@ __device__ __forceinline__ void accum_vec<float>(double* acc, const uint4& v) {
   acc[3] += static_cast<double>(__uint_as_float(v.w));
 }
 
-// grid (nb, B*H, 2): z = 0 pools qt, z = 1 pools kt. Sums in fp64 (a sum of
-// bf16 or fp32 values is exact there for any realistic spread of exponents),
-// one division by the number of real tokens. Each thread issues kPoolLoads
-// 16-byte loads before it accumulates them; few registers keep four CTAs per
-// SM in flight.
-constexpr int kPoolLoads = 4;
+// One warp per (tensor, b*h, block): z = 0 pools qt, z = 1 pools kt. Lane l
+// owns the 16-byte column vector l % vpr of the rows l / vpr, l / vpr + 32/vpr,
+// ... (a warp instruction reads 512 contiguous bytes), four loads in flight;
+// the row groups are combined with shuffles. Sums in fp64 (a sum of bf16 or
+// fp32 values is exact there for any realistic spread of exponents), one
+// division by the number of real tokens. No shared memory, no block barrier.
+constexpr int kPoolWarps = 8;
+constexpr int kPoolUnroll = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(kPoolThreads, 4)
+__global__ void __launch_bounds__(kPoolWarps * 32)
     pool_kernel(KGeom g, const char* __restrict__ qt, const char* __restrict__ kt,
                 double* __restrict__ qbar, double* __restrict__ kbar) {
   constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
-  const int j = blockIdx.x, bh = blockIdx.y;
-  const char* src = blockIdx.z == 0 ? qt : kt;
-  double* dst = blockIdx.z == 0 ? qbar : kbar;
-  const int vpr = g.d / EPV;            // vectors per row (8..32)
-  const int groups = kPoolThreads / vpr;  // row groups
-  const int c = threadIdx.x % vpr;
-  const int rg = threadIdx.x / vpr;
-
+  const int lane = threadIdx.x & 31;
+  const int64_t item = static_cast<int64_t>(blockIdx.x) * kPoolWarps + (threadIdx.x >> 5);
+  const int64_t per_tensor = static_cast<int64_t>(g.B) * g.H * g.nb;
+  if (item >= 2 * per_tensor) return;
+  const int z = item >= per_tensor ? 1 : 0;
+  const int64_t bj = item - z * per_tensor;  // (b*H + h) * nb + j
+  const int j = static_cast<int>(bj % g.nb);
+  const int64_t bh = bj / g.nb;
+  const char* src = z == 0 ? qt : kt;
+  double* dst = z == 0 ? qbar : kbar;
+  const int vpr = g.d / EPV;  // vectors per row: 8, 16 or 32
+  const int rpi = 32 / vpr;   // rows per warp instruction
+  const int c = lane % vpr, rsub = lane / vpr;
   // the block's real tokens occupy its first len slots (both orders)
   const int len = block_len(g, j);
-
   const int64_t row_bytes = static_cast<int64_t>(g.d) * sizeof(T);
-  const char* base = src + (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * row_bytes;
+  const char* base = src + (bh * g.Npad + static_cast<int64_t>(j) * g.bs) * row_bytes + c * 16;
   double acc[EPV];
 #pragma unroll
   for (int e = 0; e < EPV; ++e) acc[e] = 0.0;
-  for (int o0 = rg; o0 < len; o0 += groups * kPoolLoads) {
-    uint4 v[kPoolLoads];
+  for (int o0 = rsub; o0 < len; o0 += rpi * kPoolUnroll) {
+    uint4 v[kPoolUnroll];
 #pragma unroll
-    for (int u = 0; u < kPoolLoads; ++u) {
-      const int o = o0 + u * groups;
-      if (o < len) v[u] = __ldg(reinterpret_cast<const uint4*>(base + o * row_bytes + c * 16));
+    for (int u = 0; u < kPoolUnroll; ++u) {
+      const int o = o0 + u * rpi;
+      if (o < len) v[u] = __ldg(reinterpret_cast<const uint4*>(base + o * row_bytes));
     }
 #pragma unroll
-    for (int u = 0; u < kPoolLoads; ++u)
-      if (o0 + u * groups < len) accum_vec<T>(acc, v[u]);
+    for (int u = 0; u < kPoolUnroll; ++u)
+      if (o0 + u * rpi < len) accum_vec<T>(acc, v[u]);
   }
-  __shared__ double red[kPoolThreads * 8];
-  // red[rg][d]: reduce over row groups
+  for (int off = vpr; off < 32; off <<= 1) {
 #pragma unroll
-  for (int e = 0; e < EPV; ++e) red[rg * g.d + c * EPV + e] = acc[e];
-  __syncthreads();
-  const double dlen = static_cast<double>(len);
-  for (int col = threadIdx.x; col < g.d; col += kPoolThreads) {
-    double s = 0.0;
-    for (int r = 0; r < groups; ++r) s += red[r * g.d + col];
-    dst[(static_cast<int64_t>(bh) * g.nb + j) * g.d + col] = s / dlen;
+    for (int e = 0; e < EPV; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  }
+  if (rsub == 0) {
+    const double dlen = static_cast<double>(len);
+    double* out = dst + bj * g.d + c * EPV;
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) out[e] = acc[e] / dlen;
   }
 }
 
@@ -124,7 +118,6 @@ __global__ void __launch_bounds__(kPoolThreads, 4)
 // where the cumulative mass at the cut lies within rounding of p.
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kMaxE = 32;    // probabilities per lane (nb <= 1024)
 
 struct SelectArgs {
   float top_p[256];
@@ -145,7 +138,8 @@ __device__ __forceinline__ int warp_sum_int(int v) {
 // Pooled scores of a chunk of heads: S[bh - h0][i][j] = (Qbar_i . Kbar_j) / sqrt(d)
 // in fp64, each product summed over c = 0 .. d-1 in order. A CTA computes a
 // 64 x 64 tile of one head (thread: 4 x 4 outputs), with 16-column slices of
-// the two operands staged transposed in shared memory.
+// the two operands staged transposed in shared memory (prefetching the next
+// slice into registers measured slower: it cost a resident CTA per SM).
 // grid (ceil(nb/64), ceil(nb/64), heads in the chunk).
 constexpr int kScoreTile = 64;
 constexpr int kScoreK = 16;
@@ -153,8 +147,10 @@ constexpr int kScoreK = 16;
 __global__ void __launch_bounds__(256)
     score_kernel(KGeom g, int h0, const double* __restrict__ qbar, const double* __restrict__ kbar,
                  double* __restrict__ S) {
-  __shared__ double qs[kScoreK][kScoreTile];
-  __shared__ double ks[kScoreK][kScoreTile];
+  // one padding double per row spreads the transposed stores of a warp (8 rows
+  // x 4 columns) over more banks
+  __shared__ double qs[kScoreK][kScoreTile + 1];
+  __shared__ double ks[kScoreK][kScoreTile + 1];
   const int d = g.d, nb = g.nb;
   const int bh = h0 + static_cast<int>(blockIdx.z);
   const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
@@ -166,41 +162,42 @@ __global__ void __launch_bounds__(256)
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  // loader: thread -> (row lr, 4 columns lc..lc+3) of a 64 x 16 slice; the
-  // next slice's global loads are in flight while the current one is used
+  // loader: thread -> (row lr, 4 columns lc..lc+3) of a 64 x 16 slice
   const int lr = tid >> 2, lc = (tid & 3) * 4;
   const int iq = i0 + lr, jk = j0 + lr;
-  const double2* qrow = reinterpret_cast<const double2*>(qsrc + static_cast<int64_t>(min(iq, nb - 1)) * d + lc);
-  const double2* krow = reinterpret_cast<const double2*>(ksrc + static_cast<int64_t>(min(jk, nb - 1)) * d + lc);
-  const double2 z2 = make_double2(0.0, 0.0);
-  double2 q01 = iq < nb ? __ldg(qrow) : z2, q23 = iq < nb ? __ldg(qrow + 1) : z2;
-  double2 k01 = jk < nb ? __ldg(krow) : z2, k23 = jk < nb ? __ldg(krow + 1) : z2;
   for (int c0 = 0; c0 < d; c0 += kScoreK) {
     __syncthreads();
-    qs[lc + 0][lr] = q01.x;
-    qs[lc + 1][lr] = q01.y;
-    qs[lc + 2][lr] = q23.x;
-    qs[lc + 3][lr] = q23.y;
-    ks[lc + 0][lr] = k01.x;
-    ks[lc + 1][lr] = k01.y;
-    ks[lc + 2][lr] = k23.x;
-    ks[lc + 3][lr] = k23.y;
-    __syncthreads();
-    if (c0 + kScoreK < d) {
-      const int nx = (c0 + kScoreK) / 2;  // double2 offset of the next slice
-      q01 = iq < nb ? __ldg(qrow + nx) : z2;
-      q23 = iq < nb ? __ldg(qrow + nx + 1) : z2;
-      k01 = jk < nb ? __ldg(krow + nx) : z2;
-      k23 = jk < nb ? __ldg(krow + nx + 1) : z2;
+    {
+      double2 q01 = make_double2(0.0, 0.0), q23 = q01, k01 = q01, k23 = q01;
+      if (iq < nb) {
+        const double2* src = reinterpret_cast<const double2*>(qsrc + static_cast<int64_t>(iq) * d + c0 + lc);
+        q01 = __ldg(src);
+        q23 = __ldg(src + 1);
+      }
+      if (jk < nb) {
+        const double2* src = reinterpret_cast<const double2*>(ksrc + static_cast<int64_t>(jk) * d + c0 + lc);
+        k01 = __ldg(src);
+        k23 = __ldg(src + 1);
+      }
+      qs[lc + 0][lr] = q01.x;
+      qs[lc + 1][lr] = q01.y;
+      qs[lc + 2][lr] = q23.x;
+      qs[lc + 3][lr] = q23.y;
+      ks[lc + 0][lr] = k01.x;
+      ks[lc + 1][lr] = k01.y;
+      ks[lc + 2][lr] = k23.x;
+      ks[lc + 3][lr] = k23.y;
     }
+    __syncthreads();
 #pragma unroll
     for (int c = 0; c < kScoreK; ++c) {
-      const double2 qa = *reinterpret_cast<const double2*>(&qs[c][ty * 4]);
-      const double2 qb = *reinterpret_cast<const double2*>(&qs[c][ty * 4 + 2]);
-      const double2 ka = *reinterpret_cast<const double2*>(&ks[c][tx * 4]);
-      const double2 kb = *reinterpret_cast<const double2*>(&ks[c][tx * 4 + 2]);
-      const double qv[4] = {qa.x, qa.y, qb.x, qb.y};
-      const double kv[4] = {ka.x, ka.y, kb.x, kb.y};
+      // rows ty + 16a, columns tx + 16b: a half-warp reads 16 consecutive
+      // doubles of ks (one wavefront) and a broadcast of qs
+      double qv[4], kv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) qv[a] = qs[c][ty + 16 * a];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) kv[b] = ks[c][tx + 16 * b];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -211,11 +208,11 @@ __global__ void __launch_bounds__(256)
   double* dst = S + static_cast<int64_t>(blockIdx.z) * nb * nb;
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty * 4 + a;
+    const int i = i0 + ty + 16 * a;
     if (i >= nb) continue;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const int j = j0 + tx * 4 + b;
+      const int j = j0 + tx + 16 * b;
       if (j < nb) dst[static_cast<int64_t>(i) * nb + j] = acc[a][b] / sqrt_d;
     }
   }
@@ -227,6 +224,8 @@ __global__ void __launch_bounds__(256)
 // pattern of v (warp mass sums), the ties of v taken in index order until the
 // mass reaches p; the Top-k floor by the same bisection on counts. No sort.
 // Writes the row's bitmask words and row_cnt. grid ceil(rows of chunk / 8).
+// KE: probabilities per lane (the smallest of 8, 16, 32 with 32*KE >= nb).
+template <int KE>
 __global__ void __launch_bounds__(kSelThreads)
     cut_kernel(KGeom g, int h0, int nheads, const double* __restrict__ S, SelectArgs sa, int top_k,
                uint32_t* __restrict__ bitmask, int32_t* __restrict__ row_cnt) {
@@ -248,10 +247,10 @@ __global__ void __launch_bounds__(kSelThreads)
   const int E = (nb + 31) >> 5;
   {
     // softmax in fp64: shift by the row max, exp, divide by the sum
-    double pv[kMaxE];
+    double pv[KE];
     double mx = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < kMaxE; ++e) {
+    for (int e = 0; e < KE; ++e) {
       const int j = lane + 32 * e;
       pv[e] = (e < E && j < nb) ? __ldcg(srow + j) : -INFINITY;
       mx = fmax(mx, pv[e]);
@@ -260,16 +259,17 @@ __global__ void __launch_bounds__(kSelThreads)
     for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     double esum = 0.0;
 #pragma unroll
-    for (int e = 0; e < kMaxE; ++e) {
+    for (int e = 0; e < KE; ++e) {
       const int j = lane + 32 * e;
       pv[e] = (e < E && j < nb) ? exp(pv[e] - mx) : 0.0;
       esum += pv[e];
     }
     esum = warp_sum(esum);
+    const double inv = 1.0 / esum;  // one division per row
 #pragma unroll
-    for (int e = 0; e < kMaxE; ++e) {
+    for (int e = 0; e < KE; ++e) {
       const int j = lane + 32 * e;
-      pv[e] = (e < E && j < nb) ? pv[e] / esum : -1.0;  // -1: not a key block
+      pv[e] = (e < E && j < nb) ? pv[e] * inv : -1.0;  // -1: not a key block
     }
     // mass and count of the row's probabilities >= v (the -1 entries never
     // pass: every v tried is a non-negative double, bit 62 of its pattern
@@ -278,8 +278,28 @@ __global__ void __launch_bounds__(kSelThreads)
       double mm = 0.0;
       int cc = 0;
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e)
+      for (int e = 0; e < KE; ++e)
         if (e < E && pv[e] >= v) {
+          mm += pv[e];
+          ++cc;
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mm += __shfl_xor_sync(0xffffffffu, mm, o);
+        cc += __shfl_xor_sync(0xffffffffu, cc, o);
+      }
+      m = mm;
+      c = cc;
+    };
+    // the same for a threshold whose low 32 bits are zero: the comparison of
+    // two non-negative doubles is that of their bit patterns, so the high
+    // words decide it (an integer compare; the -1 entries are negative)
+    auto ge_sums_hi = [&](int vhi, double& m, int& c) {
+      double mm = 0.0;
+      int cc = 0;
+#pragma unroll
+      for (int e = 0; e < KE; ++e)
+        if (e < E && __double2hiint(pv[e]) >= vhi) {
           mm += pv[e];
           ++cc;
         }
@@ -298,7 +318,7 @@ __global__ void __launch_bounds__(kSelThreads)
       double f = -1.0;
       const double a = as_double(lo), b = as_double(hi);
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e)
+      for (int e = 0; e < KE; ++e)
         if (e < E && pv[e] >= a && pv[e] < b) f = pv[e];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) f = fmax(f, __shfl_xor_sync(0xffffffffu, f, o));
@@ -320,7 +340,10 @@ __global__ void __launch_bounds__(kSelThreads)
       for (; b >= 0 && c_lo - c_hi > 32; --b) {
         const unsigned long long mid = lo | (1ull << b);
         int c;
-        ge_sums(as_double(mid), m, c);
+        if (b >= 32)  // lo and mid have zero low words
+          ge_sums_hi(static_cast<int>(mid >> 32), m, c);
+        else
+          ge_sums(as_double(mid), m, c);
         const bool ok = by_mass ? (m >= p_or_n) : (static_cast<double>(c) >= p_or_n);
         if (ok) {
           lo = mid;
@@ -336,7 +359,7 @@ __global__ void __launch_bounds__(kSelThreads)
       const double a = as_double(lo), bv = as_double(hi);
       int mine = 0;
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e)
+      for (int e = 0; e < KE; ++e)
         if (e < E && pv[e] >= a && pv[e] < bv) ++mine;
       int incl = mine;
 #pragma unroll
@@ -347,7 +370,7 @@ __global__ void __launch_bounds__(kSelThreads)
       int slot = incl - mine;
       __syncwarp();
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e)
+      for (int e = 0; e < KE; ++e)
         if (e < E && pv[e] >= a && pv[e] < bv) cbuf[slot++] = pv[e];
       __syncwarp();
       const double cand = lane < c_lo - c_hi ? cbuf[lane] : -1.0;
@@ -396,7 +419,7 @@ __global__ void __launch_bounds__(kSelThreads)
       int c_gt = 0, c_eq = 0;
       const double vT = as_double(T);
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e) {
+      for (int e = 0; e < KE; ++e) {
         if (e < E) {
           if (pv[e] > vT) {
             m_gt += pv[e];
@@ -432,7 +455,7 @@ __global__ void __launch_bounds__(kSelThreads)
       const double vT = as_double(T);
       int c_gt = 0;
 #pragma unroll
-      for (int e = 0; e < kMaxE; ++e)
+      for (int e = 0; e < KE; ++e)
         if (e < E && pv[e] > vT) ++c_gt;
       c_gt = warp_sum_int(c_gt);
       vsel = T;
@@ -447,7 +470,7 @@ __global__ void __launch_bounds__(kSelThreads)
     int before = 0;  // ties of vsel at lower indices
     uint32_t myword = 0u;
 #pragma unroll
-    for (int e = 0; e < kMaxE; ++e) {
+    for (int e = 0; e < KE; ++e) {
       if (e < E) {
         const bool real = pv[e] >= 0.0;
         bool keep;
@@ -662,13 +685,14 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
   KGeom g = make_kgeom(p);
   const int BH = g.B * g.H;
 
-  dim3 pg(g.nb, BH, 2);
+  const int64_t pool_items = 2ll * BH * g.nb;
+  const unsigned pg = static_cast<unsigned>((pool_items + kPoolWarps - 1) / kPoolWarps);
   if (p->g.dtype == SBA_BF16)
-    pool_kernel<__nv_bfloat16><<<pg, kPoolThreads, 0, st>>>(g, static_cast<const char*>(qt),
-                                                            static_cast<const char*>(kt), qbar, kbar);
+    pool_kernel<__nv_bfloat16><<<pg, kPoolWarps * 32, 0, st>>>(g, static_cast<const char*>(qt),
+                                                               static_cast<const char*>(kt), qbar, kbar);
   else
-    pool_kernel<float><<<pg, kPoolThreads, 0, st>>>(g, static_cast<const char*>(qt),
-                                                    static_cast<const char*>(kt), qbar, kbar);
+    pool_kernel<float><<<pg, kPoolWarps * 32, 0, st>>>(g, static_cast<const char*>(qt),
+                                                       static_cast<const char*>(kt), qbar, kbar);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -683,8 +707,13 @@ cudaError_t launch_build_mask(const sba_plan* p, const void* qt, const void* kt,
   for (int h0 = 0; h0 < BH; h0 += hc) {
     const int nh = std::min(hc, BH - h0);
     score_kernel<<<dim3(nt, nt, nh), 256, 0, st>>>(g, h0, qbar, kbar, scores);
-    cut_kernel<<<(nh * g.nb + kSelWarps - 1) / kSelWarps, kSelThreads, 0, st>>>(
-        g, h0, nh, scores, sa, top_k, bitmask, row_cnt);
+    const unsigned cg = static_cast<unsigned>((nh * g.nb + kSelWarps - 1) / kSelWarps);
+    if (g.nb <= 256)
+      cut_kernel<8><<<cg, kSelThreads, 0, st>>>(g, h0, nh, scores, sa, top_k, bitmask, row_cnt);
+    else if (g.nb <= 512)
+      cut_kernel<16><<<cg, kSelThreads, 0, st>>>(g, h0, nh, scores, sa, top_k, bitmask, row_cnt);
+    else
+      cut_kernel<32><<<cg, kSelThreads, 0, st>>>(g, h0, nh, scores, sa, top_k, bitmask, row_cnt);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

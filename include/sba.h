@@ -308,13 +308,18 @@ SBA_API sba_status sba_attention_lowbit(const sba_plan* plan, const void* qt, co
  *   row_ptr, col_idx  the CSR from sba_build_mask (or any CSR over [0, nb)
  *                     with at most nb columns per row)
  *   work_order        int32 [R], required for SBA_SCHED_LPT, ignored (may be
- *                     NULL) for SBA_SCHED_HEAD_MAJOR
+ *                     NULL) for SBA_SCHED_HEAD_MAJOR. bf16 plans with bs = 64
+ *                     run pairs of query blocks (2i, 2i+1) of a head as one
+ *                     128-row tile over the union of their columns, taken in
+ *                     head order; work_order is then not read (it must still
+ *                     be non-NULL for SBA_SCHED_LPT)
  *   lse               float [B][H][Npad] or NULL
  *   trace             NULL, or uint64 [R][3] receiving, per row, the
  *                     %globaltimer ns at which its CTA started and finished it
  *                     and the SM id (for the SM idle / tail measurement)
- * A column index outside [0, nb) is replaced by 0 and flags
- * SBA_ERR_DEVICE_CHECK in the workspace status word. */
+ * A column index outside [0, nb) is replaced by 0, and a row whose row_ptr
+ * range is negative, longer than nb or past B*H*nb*nb is skipped (written as
+ * empty); both flag SBA_ERR_DEVICE_CHECK in the workspace status word. */
 SBA_API sba_status sba_attention(const sba_plan* plan, const void* qt, const void* kt, const void* vt,
                          const int32_t* row_ptr, const int32_t* col_idx,
                          const int32_t* work_order, void* ot, float* lse,
