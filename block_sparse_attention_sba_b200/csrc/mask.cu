@@ -331,16 +331,41 @@ __global__ void __launch_bounds__(kSelThreads)
     // Once at most 32 elements are left in [lo, hi) they are gathered one per
     // lane (through this warp's slice of shared memory) and the remaining
     // steps sum only them on top of the mass and count at hi.
+    // the row's smallest and largest probability, as bit patterns
+    unsigned long long pat_min, pat_max;
+    {
+      double pmin = 2.0, pmax = 0.0;
+#pragma unroll
+      for (int e = 0; e < KE; ++e)
+        if (e < E && pv[e] >= 0.0) {
+          pmin = fmin(pmin, pv[e]);
+          pmax = fmax(pmax, pv[e]);
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        pmin = fmin(pmin, __shfl_xor_sync(0xffffffffu, pmin, o));
+        pmax = fmax(pmax, __shfl_xor_sync(0xffffffffu, pmax, o));
+      }
+      pat_min = static_cast<unsigned long long>(__double_as_longlong(pmin));
+      pat_max = static_cast<unsigned long long>(__double_as_longlong(pmax));
+    }
+    double total;
+    int cnt_all;
+    ge_sums(0.0, total, cnt_all);
     auto bisect = [&](bool by_mass, double p_or_n) -> unsigned long long {
-      unsigned long long lo = 0ull, hi = 1ull << 62;
+      // start from the row's own range: lo = the common bit prefix of its
+      // smallest and largest probability (every element is >= lo), hi = lo
+      // plus one unit of the highest bit where they differ (> the largest)
+      const unsigned long long diff = pat_min ^ pat_max;
+      int b = diff ? 63 - __clzll(static_cast<long long>(diff)) : -1;
+      const unsigned long long span = b >= 0 ? (1ull << (b + 1)) : 1ull;
+      unsigned long long lo = pat_min & ~(span - 1ull), hi = lo + span;
       double m, m_hi = 0.0;
-      int c_lo, c_hi = 0;
-      ge_sums(0.0, m, c_lo);
-      int b = 61;
+      int c_lo = cnt_all, c_hi = 0;
       for (; b >= 0 && c_lo - c_hi > 32; --b) {
         const unsigned long long mid = lo | (1ull << b);
         int c;
-        if (b >= 32)  // lo and mid have zero low words
+        if ((mid & 0xffffffffull) == 0ull)  // the high words decide
           ge_sums_hi(static_cast<int>(mid >> 32), m, c);
         else
           ge_sums(as_double(mid), m, c);
@@ -409,9 +434,6 @@ __global__ void __launch_bounds__(kSelThreads)
     unsigned long long vsel = 0ull;  // the value at the cut
     int take = 0;                    // ties of vsel taken, lowest index first
     bool have_cut = false;
-    double total;
-    int cnt_all;
-    ge_sums(0.0, total, cnt_all);
     if (p < 1.0 && total >= p) {
       const unsigned long long T = bisect(true, p);
       // elements above the cut, then ties of the cut value one at a time
