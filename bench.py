@@ -73,8 +73,13 @@ def _config(wl, extra=None):
 
 
 def _block_lens(wl):
-    """Real tokens per block (for the valid-FLOP count), row-major over cubes."""
+    """Real tokens per block (for the valid-FLOP count): row-major over cubes,
+    or, in Hilbert order, full blocks but the last."""
     ct, ch, cw = wl.cube
+    if getattr(wl, "order", "cube") == "hilbert":
+        bs, N = ct * ch * cw, wl.T * wl.Hh * wl.W
+        nb = -(-N // bs)
+        return [bs] * (nb - 1) + [N - (nb - 1) * bs]
     nT, nH, nW = -(-wl.T // ct), -(-wl.Hh // ch), -(-wl.W // cw)
     lens = []
     for tt in range(nT):
