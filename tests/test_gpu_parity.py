@@ -34,9 +34,15 @@ SMALL = {
     "hilbert_f32": datagen.custom("hilbert_f32", 1, 2, 5, 6, 7, 64, (4, 4, 4), dtype="f32",
                                   top_p=(0.9,), top_k=1, order="hilbert"),
     # 1080 rows (40 heads x 27 blocks, ragged in h and w): several rows per
-    # persistent CTA, so both query tiles of a CTA go through row changes
+    # persistent CTA, so a CTA goes through many row changes
     "many_rows_d128": datagen.custom("many_rows_d128", 1, 40, 6, 22, 21, 128, (2, 8, 8),
                                      top_p=(0.5, 0.9, 0.97), top_k=2, rope_split=(44, 42, 42)),
+    # block size 64 with an odd number of blocks per head (27): the last pair
+    # of query blocks has no second block; corner cubes hold a single token
+    "pairs_odd_bs64": datagen.custom("pairs_odd_bs64", 1, 2, 3, 17, 17, 128, (1, 8, 8),
+                                     top_p=(0.7, 0.9), top_k=2, rope_split=(44, 42, 42)),
+    "pairs_odd_d64": datagen.custom("pairs_odd_d64", 2, 2, 9, 12, 12, 64, (4, 4, 4),
+                                    top_p=(0.6, 0.95), top_k=1, rope_split=(16, 24, 24)),
 }
 
 
@@ -178,7 +184,8 @@ def _attn_with_csr(wl, q, k, v, row_ptr, col_idx, sched=1, work_counts=None):
     return sa, sa.check()
 
 
-@pytest.mark.parametrize("name", ["ragged_d128_bs64", "ragged_d128_bs128", "ragged_d64_bs128"])
+@pytest.mark.parametrize("name", ["ragged_d128_bs64", "pairs_odd_bs64", "ragged_d128_bs128",
+                                  "ragged_d64_bs128"])
 @pytest.mark.parametrize("sched", [0, 1])
 def test_handmade_csr_with_empty_and_single_block_rows(sched, name):
     wl = SMALL[name]
