@@ -104,6 +104,9 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_O = 384;
   static constexpr uint32_t IDESC_MEAN = idesc_tf32_f32(M, D);
+  // (the low-bit constants are referenced here so that the bf16
+  // instantiations, which do not use them, compile without warnings)
+  static_assert(LB_BIAS > 0.0f && RESCALE > 0.0f && IDESC_MEAN != 0u, "low-bit constants");
   // barrier indices
   static constexpr int B_QF = 0, B_QE = 1, B_KF = 2, B_KE = B_KF + NK, B_VF = B_KE + NK,
                        B_VE = B_VF + NV, B_SR = B_VE + NV, B_PR = B_SR + NSB, B_PD = B_PR + NSB,

@@ -129,11 +129,8 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
-__device__ __forceinline__ int warp_sum_int(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
+// (one warp-wide reduction instruction)
+__device__ __forceinline__ int warp_sum_int(int v) { return __reduce_add_sync(0xffffffffu, v); }
 
 // Pooled scores of a chunk of heads: S[bh - h0][i][j] = (Qbar_i . Kbar_j) / sqrt(d)
 // in fp64, each product summed over c = 0 .. d-1 in order. A CTA computes a
@@ -283,13 +280,8 @@ __global__ void __launch_bounds__(kSelThreads)
           mm += pv[e];
           ++cc;
         }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mm += __shfl_xor_sync(0xffffffffu, mm, o);
-        cc += __shfl_xor_sync(0xffffffffu, cc, o);
-      }
-      m = mm;
-      c = cc;
+      m = warp_sum(mm);
+      c = warp_sum_int(cc);
     };
     // the same for a threshold whose low 32 bits are zero: the comparison of
     // two non-negative doubles is that of their bit patterns, so the high
@@ -303,13 +295,8 @@ __global__ void __launch_bounds__(kSelThreads)
           mm += pv[e];
           ++cc;
         }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mm += __shfl_xor_sync(0xffffffffu, mm, o);
-        cc += __shfl_xor_sync(0xffffffffu, cc, o);
-      }
-      m = mm;
-      c = cc;
+      m = warp_sum(mm);
+      c = warp_sum_int(cc);
     };
     auto as_double = [](unsigned long long b) { return __longlong_as_double(static_cast<long long>(b)); };
     // The single probability in [lo, hi) (bit patterns), found once the
@@ -400,32 +387,24 @@ __global__ void __launch_bounds__(kSelThreads)
       __syncwarp();
       const double cand = lane < c_lo - c_hi ? cbuf[lane] : -1.0;
       __syncwarp();
-      for (; b >= 0 && c_lo - c_hi > 1; --b) {
-        const unsigned long long mid = lo | (1ull << b);
-        const double vm = as_double(mid);
-        // only the candidates still in [mid, hi): those at or above hi are in
-        // the mass and count at hi already
-        const bool in = cand >= vm && cand < as_double(hi);
-        const int c = c_hi + __popc(__ballot_sync(0xffffffffu, in));
-        m = m_hi + warp_sum(in ? cand : 0.0);
-        const bool ok = by_mass ? (m >= p_or_n) : (static_cast<double>(c) >= p_or_n);
-        if (ok) {
-          lo = mid;
-          c_lo = c;
-        } else {
-          hi = mid;
-          c_hi = c;
-          m_hi = m;
+      // every candidate against every other: the mass and count of the
+      // probabilities >= each candidate (those at or above hi are in m_hi,
+      // c_hi); the answer is the largest candidate whose predicate holds
+      double am = 0.0;
+      int ac = 0;
+#pragma unroll 4
+      for (int jl = 0; jl < 32; ++jl) {
+        const double v = __shfl_sync(0xffffffffu, cand, jl);
+        if (v >= cand) {
+          am += v;
+          ++ac;
         }
       }
-      if (c_lo - c_hi == 1) {
-        const double lo_v = as_double(lo), hi_v = as_double(hi);
-        double f = (cand >= lo_v && cand < hi_v) ? cand : -1.0;
+      const bool ok = by_mass ? (m_hi + am >= p_or_n) : (static_cast<double>(c_hi + ac) >= p_or_n);
+      double f = (ok && cand >= 0.0) ? cand : -1.0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) f = fmax(f, __shfl_xor_sync(0xffffffffu, f, o));
-        return static_cast<unsigned long long>(__double_as_longlong(f));
-      }
-      return lo;
+      for (int o = 16; o > 0; o >>= 1) f = fmax(f, __shfl_xor_sync(0xffffffffu, f, o));
+      return static_cast<unsigned long long>(__double_as_longlong(f));
     };
     // Top-p: n_p = the length of the shortest prefix, in descending order
     // (ties: lower index first), whose cumulative mass reaches p; all blocks
