@@ -144,6 +144,8 @@ class HeadShardedAttention:
         self.pg = pg
         self.world = dist.get_world_size(pg)
         self.rank = dist.get_rank(pg)
+        if H < self.world:
+            raise ValueError(f"{H} heads on {self.world} ranks: every rank must start with a head")
         self.store = store
         self.checkin_timeout = datetime.timedelta(seconds=checkin_timeout_s)
         self.step_no = 0

@@ -42,6 +42,21 @@ def test_lpt_placement_is_longest_first_and_within_grahams_bound():
     assert lpt_placement([5, 1, 1, 1, 1, 1], 2) == [0, 1, 1, 1, 1, 1]
 
 
+def test_fewer_heads_than_ranks_is_rejected():
+    import datetime
+    import torch.distributed as dist
+    from block_sparse_attention_sba_b200.sharded import HeadShardedAttention
+    store = dist.HashStore()
+    dist.init_process_group("gloo", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=10))
+    try:
+        HeadShardedAttention(object(), 1, dist.group.WORLD)  # 1 head, 1 rank: fine
+        with pytest.raises(ValueError):
+            HeadShardedAttention(object(), 0, dist.group.WORLD)
+    finally:
+        dist.destroy_process_group()
+
+
 def test_static_split_and_moves():
     assert static_heads(5, 2, 0) == [0, 2, 4] and static_heads(5, 2, 1) == [1, 3]
     assert migrations([0, 1, 0, 0, 1], 2) == [(3, 1, 0), (4, 0, 1)]
