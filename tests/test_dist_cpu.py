@@ -75,3 +75,21 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     args = types.SimpleNamespace(workload="wan", steps=1, warmup=0, gpus=2)
     assert bench.run_reference(args) == 0  # returns at once, no data generated
+
+
+def test_block_lengths_count_every_real_token_once():
+    """The bench's real-token FLOP count: block lengths sum to N in both
+    orders, cube order follows the grid's edge cubes, Hilbert order has full
+    blocks but the last (checked against the oracle's own lengths)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import datagen
+    import numpy as np
+    import oracle
+    for wl in (datagen.WORKLOADS["wan"], datagen.WORKLOADS["small"],
+               datagen.with_order(datagen.WORKLOADS["wan"], "hilbert"),
+               datagen.custom("odd", 1, 1, 3, 17, 17, 128, (1, 8, 8))):
+        lens = bench._block_lens(wl)
+        g = oracle.Geom(wl.T, wl.Hh, wl.W, *wl.cube, order=getattr(wl, "order", "cube"))
+        assert sum(lens) == wl.T * wl.Hh * wl.W
+        assert np.array_equal(np.array(lens), oracle.block_len(g))
