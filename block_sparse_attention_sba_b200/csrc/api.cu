@@ -207,7 +207,8 @@ sba_status sba_plan_create(const sba_geometry* geom, sba_plan** out) {
     p->info.workspace_bytes += align256(static_cast<size_t>(Npad) * sizeof(int32_t));
   }
   p->ws_heads = p->info.workspace_bytes;
-  p->info.workspace_bytes += align256(static_cast<size_t>(G.B) * G.H * sizeof(uint32_t));
+  // V-Smooth's per-head words: completed-statistics counts, then maxima
+  p->info.workspace_bytes += align256(2 * static_cast<size_t>(G.B) * G.H * sizeof(uint32_t));
   p->wait_budget_ns = 4000000000ull;  // 4 s: no healthy wait comes near it
   const char* env = getenv("SBA_WAIT_BUDGET_NS");
   if (env) {
@@ -233,7 +234,7 @@ sba_status sba_workspace_init(const sba_plan* plan, void* workspace, void* strea
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(Ctrl), st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   e = cudaMemsetAsync(static_cast<char*>(workspace) + plan->ws_heads, 0,
-                      static_cast<size_t>(plan->g.B) * plan->g.H * sizeof(uint32_t), st);
+                      2 * static_cast<size_t>(plan->g.B) * plan->g.H * sizeof(uint32_t), st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   if (plan->g.order == SBA_ORDER_HILBERT) {
     // from pageable host memory: returns once the table has been staged

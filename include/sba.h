@@ -267,7 +267,8 @@ SBA_API sba_status sba_build_stripe_mask(const sba_plan* plan, const sba_stripe*
  * Outputs (device, caller-owned): vq uint8 [B][H][nb][d][bs] - each block's
  *   codes transposed, channel-major (16-byte aligned); vmean fp32
  *   [B][H][nb][d] (16-byte aligned); vexp int32 [B][H]. workspace as for
- *   sba_build_mask (its pooled-means area holds per-block maxima meanwhile).
+ *   sba_build_mask (two per-head words in it count finished blocks and hold
+ *   the head's maximum meanwhile; zero again when the call completes).
  * bf16 plans with d <= 128 only (else SBA_ERR_UNSUPPORTED). Deterministic. */
 SBA_API sba_status sba_smooth_v(const sba_plan* plan, const void* vt, void* vq, float* vmean,
                                 int32_t* vexp, void* workspace, void* stream);
