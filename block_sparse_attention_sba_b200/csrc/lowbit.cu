@@ -91,186 +91,246 @@ __device__ __forceinline__ void smooth_item(uint32_t item, int nb, int BH, int L
   }
 }
 
-__device__ __forceinline__ float block_max_f(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float m = red[0];
-#pragma unroll
-  for (int w = 1; w < kSmoothThreads / 32; ++w) m = fmaxf(m, red[w]);
-  return m;
-}
+constexpr int kSmoothBufs = 2;  // blocks staged per CTA
 
-// Per-channel means of the staged block's len real rows into smu[0..d):
-// thread = (channel pair, row group), fp64 sums, one division, one rounding
-// to fp32. Deterministic: both item kinds get the same bits.
-__device__ __forceinline__ void block_means(const __nv_bfloat162* b2, int len, int d, double* dsum,
-                                            float* smu) {
-  const int tid = threadIdx.x, npair = d / 2, groups = kSmoothThreads / npair;
-  const int cp = tid % npair, rg = tid / npair;
-  double s0 = 0.0, s1 = 0.0;
-  for (int o = rg; o < len; o += groups) {
-    const float2 f = __bfloat1622float2(b2[o * npair + cp]);
-    s0 += static_cast<double>(f.x);
-    s1 += static_cast<double>(f.y);
-  }
-  dsum[2 * tid] = s0;
-  dsum[2 * tid + 1] = s1;
-  __syncthreads();
-  if (tid < d) {
-    double t = 0.0;
-    for (int r = 0; r < groups; ++r) t += dsum[2 * (r * npair + tid / 2) + (tid & 1)];
-    smu[tid] = static_cast<float>(t / static_cast<double>(len));
-  }
-  __syncthreads();
-}
+// Per staged block: the item, and for a quantisation item the head's e.
+struct SmoothSlot {
+  uint32_t item;
+  int32_t e;
+};
 
-__global__ void __launch_bounds__(kSmoothThreads)
+// Warp roles: warps 0..7 process blocks (kSmoothThreads threads), warp 8
+// produces: it takes items from the counter, resolves a quantisation item's
+// dependency (the head's statistics complete), reads the head's exponent and
+// the block's means, and stages the block with one bulk copy into a ring of
+// kSmoothBufs buffers (full / empty mbarriers).
+//
+// Statistics item, one pass over the staged block: per channel the fp64 sum
+// and the fp32 minimum and maximum over the real rows (thread = channel pair x
+// row group, rows strided by the group count), combined in group order.
+// mu = fp32(sum / len); max |R| over the block = max(vmax - mu, mu - vmin) in
+// fp32 (rounding is monotone, so the largest |fl(v - mu)| is at the largest
+// or the smallest v).
+// Quantisation item, one pass: thread = 4 channels x 16 rows; codes of one
+// channel's 16 rows are one 16-byte store.
+__global__ void __launch_bounds__(kSmoothThreads + 32)
     smooth_v_kernel(KGeom g, SmoothArgs a) {
-  extern __shared__ __align__(128) unsigned char sm_raw[];  // two [bs][d] bf16 buffers
-  __shared__ double dsum[2 * kSmoothThreads];
+  extern __shared__ __align__(128) unsigned char sm_raw[];  // [bufs][bs][d] bf16, then [bufs][d] f32
+  // groups * d = 512 for d = 64 and 128 (groups = 2 * kSmoothThreads / d)
+  __shared__ double dsum[512];                // [groups][d] partial sums
+  __shared__ float dmin[512], dmax[512];      // [groups][d] partial minima / maxima
   __shared__ float red[kSmoothThreads / 32];
-  __shared__ float smu[128];
-  __shared__ __align__(8) uint64_t bars[2];
-  __shared__ uint32_t s_item[2];
-  __shared__ int s_abort, s_e;
+  __shared__ __align__(8) uint64_t full[kSmoothBufs], empty[kSmoothBufs];
+  __shared__ SmoothSlot slot[kSmoothBufs];
+  __shared__ int s_abort;
   const int tid = threadIdx.x, d = g.d, nb = g.nb;
   const int BH = g.B * g.H;
-  const int npair = d / 2;
   const uint32_t n_items = 2u * static_cast<uint32_t>(BH) * static_cast<uint32_t>(nb);
   const uint32_t buf_bytes = static_cast<uint32_t>(g.bs * d * 2);
+  float* means = reinterpret_cast<float*>(sm_raw + kSmoothBufs * buf_bytes);
   uint32_t* status = &a.ctrl->status;
   uint32_t* head_max = a.heads + BH;
-  // thread 0: uses of each buffer issued and waited for (a copy still in
-  // flight when the loop ends early is waited for before the CTA exits)
-  uint32_t issued0 = 0u, issued1 = 0u, waited0 = 0u, waited1 = 0u;
-  auto issue = [&](uint32_t it, int b) {
-    bool qq;
-    int bh, j;
-    smooth_item(it, nb, BH, a.lag, qq, bh, j);
-    const uint32_t bytes = static_cast<uint32_t>(block_len(g, j) * d * 2);
-    const __nv_bfloat16* src = a.vt + (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * d;
-    const uint32_t bar = smem_u32(&bars[b]);
-    fence_proxy_async_smem();  // the buffer's previous reads come first
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_load_1d(smem_u32(sm_raw + b * buf_bytes), src, bytes, bar);
-    if (b) ++issued1; else ++issued0;
-  };
+  volatile int* abort_flag = &s_abort;
   if (tid == 0) {
-    mbar_init(smem_u32(&bars[0]), 1);
-    mbar_init(smem_u32(&bars[1]), 1);
+    for (int b = 0; b < kSmoothBufs; ++b) {
+      mbar_init(smem_u32(&full[b]), 1);
+      mbar_init(smem_u32(&empty[b]), kSmoothThreads / 32);
+    }
     fence_barrier_init();
     s_abort = 0;
-    const uint32_t first = atomicAdd(&a.ctrl->aux_next, 1u);
-    s_item[0] = first;
-    if (first < n_items) issue(first, 0);
   }
   __syncthreads();
-  for (uint32_t k = 0;; ++k) {
-    const int buf = static_cast<int>(k & 1u);
-    const uint32_t item = s_item[buf];
-    if (item >= n_items) break;
-    if (tid == 0) {
-      // take the next item and start its copy into the other buffer (free:
-      // the previous item's reads ended at its closing barrier)
-      const uint32_t next = atomicAdd(&a.ctrl->aux_next, 1u);
-      s_item[buf ^ 1] = next;
-      if (next < n_items) issue(next, buf ^ 1);
-    }
-    bool quant;
-    int bh, j;
-    smooth_item(item, nb, BH, a.lag, quant, bh, j);
-    const int len = block_len(g, j);
-    const bool got = mbar_wait(smem_u32(&bars[buf]), (k >> 1) & 1u, a.budget_ns, &s_abort, status);
-    if (tid == 0 && got) {
-      if (buf) ++waited1; else ++waited0;
-    }
-    __syncthreads();
-    if (s_abort) break;
-    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(sm_raw + buf * buf_bytes);
-    block_means(b2, len, d, dsum, smu);
-    const int cp = tid % npair, rg = tid / npair, groups = kSmoothThreads / npair;
-    if (!quant) {
-      if (tid < d) a.vmean[(static_cast<int64_t>(bh) * nb + j) * d + tid] = smu[tid];
-      const float mu0 = smu[2 * cp], mu1 = smu[2 * cp + 1];
-      float amax = 0.f;
-      for (int o = rg; o < len; o += groups) {
-        const float2 f = __bfloat1622float2(b2[o * npair + cp]);
-        amax = fmaxf(amax, fmaxf(fabsf(f.x - mu0), fabsf(f.y - mu1)));
-      }
-      amax = block_max_f(amax, red);
-      if (tid == 0) {
-        // non-negative floats order like their bit patterns
-        atomicMax(head_max + bh, __float_as_uint(amax));
-        __threadfence();  // means and maximum before the count (after the barrier above)
-        atomicAdd(a.heads + bh, 1u);
-      }
-    } else {
-      if (tid == 0) {
-        // wait until every statistics item of the head is done
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu(a.heads + bh) < static_cast<uint32_t>(nb)) {
-          if (globaltimer_ns() - t0 > a.budget_ns) {
-            atomicOr(status, kStatusTimeout);
-            break;
-          }
-          __nanosleep(128);
-        }
-        const int e = scale_exponent(__uint_as_float(ld_acquire_gpu(head_max + bh)));
-        s_e = e;
-        if (j == 0) a.vexp[bh] = e;
-      }
-      __syncthreads();
-      const float inv = ldexpf(1.0f, -s_e);  // exact power of two
-      // 32 codes of two channels per thread: one 32-byte sector per channel
-      uint8_t* dst = a.vq + (static_cast<int64_t>(bh) * nb + j) * d * g.bs;
-      const int nhg = g.bs / 32;
-      for (int idx = tid; idx < npair * nhg; idx += kSmoothThreads) {
-        const int c2 = idx % npair, hg = idx / npair;
-        const float mu0 = smu[2 * c2], mu1 = smu[2 * c2 + 1];
-        uint32_t w0[8], w1[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float x0[4], x1[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int o = hg * 32 + 4 * q + u;
-            if (o < len) {
-              const float2 f = __bfloat1622float2(b2[o * npair + c2]);
-              x0[u] = (f.x - mu0) * inv;
-              x1[u] = (f.y - mu1) * inv;
-            } else {
-              x0[u] = 0.f;
-              x1[u] = 0.f;
+  if (tid >= kSmoothThreads) {
+    // ---------------------------------------------------------- producer
+    const int lane = tid & 31;
+    uint32_t issued = 0;  // ring uses issued (lane 0)
+    for (uint32_t k = 0;; ++k) {
+      const int b = static_cast<int>(k % kSmoothBufs);
+      const uint32_t use = k / kSmoothBufs;
+      uint32_t item = 0;
+      if (lane == 0) item = atomicAdd(&a.ctrl->aux_next, 1u);
+      item = __shfl_sync(0xffffffffu, item, 0);
+      bool quant = false;
+      int bh = 0, j = 0, e = 0;
+      if (item < n_items) {
+        smooth_item(item, nb, BH, a.lag, quant, bh, j);
+        if (quant && lane == 0) {
+          // every statistics item of the head done (bounded wait)
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(a.heads + bh) < static_cast<uint32_t>(nb)) {
+            if (*abort_flag) break;
+            if (globaltimer_ns() - t0 > a.budget_ns) {
+              atomicOr(status, kStatusTimeout);
+              *abort_flag = 1;
+              break;
             }
+            __nanosleep(64);
           }
-          w0[q] = e4m3x2(x0[0], x0[1]) | (e4m3x2(x0[2], x0[3]) << 16);
-          w1[q] = e4m3x2(x1[0], x1[1]) | (e4m3x2(x1[2], x1[3]) << 16);
+          e = scale_exponent(__uint_as_float(ld_acquire_gpu(head_max + bh)));
         }
-        uint4* p0 = reinterpret_cast<uint4*>(dst + static_cast<int64_t>(2 * c2) * g.bs + hg * 32);
-        uint4* p1 = reinterpret_cast<uint4*>(dst + static_cast<int64_t>(2 * c2 + 1) * g.bs + hg * 32);
-        p0[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-        p0[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
-        p1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-        p1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+        __syncwarp();
       }
+      // the buffer's previous block processed (bounded wait)
+      bool ok = true;
+      if (use > 0) ok = mbar_wait(smem_u32(&empty[b]), (use - 1) & 1u, a.budget_ns, abort_flag, status);
+      // leave together (the lanes below exchange values)
+      if (__any_sync(0xffffffffu, !ok || *abort_flag)) break;
+      if (item < n_items && quant) {
+        // the block's means (written before the head's count moved)
+        const float* src = a.vmean + (static_cast<int64_t>(bh) * nb + j) * d;
+        for (int c = lane; c < d / 4; c += 32)
+          reinterpret_cast<float4*>(means + b * d)[c] = __ldcg(reinterpret_cast<const float4*>(src) + c);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        slot[b].item = item < n_items ? item : n_items;
+        slot[b].e = e;
+        const uint32_t bar = smem_u32(&full[b]);
+        if (item < n_items) {
+          const uint32_t bytes = static_cast<uint32_t>(block_len(g, j) * d * 2);
+          const __nv_bfloat16* src =
+              a.vt + (static_cast<int64_t>(bh) * g.Npad + static_cast<int64_t>(j) * g.bs) * d;
+          fence_proxy_async_smem();  // the buffer's previous reads come first
+          mbar_arrive_expect_tx(bar, bytes);
+          bulk_load_1d(smem_u32(sm_raw + b * buf_bytes), src, bytes, bar);
+          ++issued;
+        } else {
+          mbar_arrive(bar);  // end of work: the consumers see the sentinel
+        }
+      }
+      if (item >= n_items) break;
     }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    // copies still in flight (only after a timed-out wait): bounded wait
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const uint32_t iss = b ? issued1 : issued0, wt = b ? waited1 : waited0;
-      if (iss > wt) {
+    if (lane == 0 && *abort_flag) {
+      // copies possibly in flight after an abort: bounded wait for the last
+      // issued use of each buffer
+      for (uint32_t u = (issued > kSmoothBufs ? issued - kSmoothBufs : 0u); u < issued; ++u) {
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(smem_u32(&bars[b]), (iss - 1u) & 1u) &&
+        while (!mbar_try_wait(smem_u32(&full[u % kSmoothBufs]), (u / kSmoothBufs) & 1u) &&
                globaltimer_ns() - t0 < a.budget_ns) {
         }
       }
     }
+  } else {
+    // --------------------------------------------------------- consumers
+    const int warp = tid >> 5, lane = tid & 31;
+    const int npair = d / 2, groups = kSmoothThreads / npair;
+    const int nq = d / 4, nrg = g.bs / 16;
+    for (uint32_t k = 0;; ++k) {
+      const int b = static_cast<int>(k % kSmoothBufs);
+      const uint32_t use = k / kSmoothBufs;
+      const bool got = mbar_wait(smem_u32(&full[b]), use & 1u, a.budget_ns, abort_flag, status);
+      // every consumer takes the same decision (the statistics path below
+      // has named barriers that need all of them)
+      if (named_bar_or(2, kSmoothThreads, !got || *abort_flag)) break;
+      const uint32_t item = slot[b].item;
+      if (item >= n_items) break;
+      bool quant;
+      int bh, j;
+      smooth_item(item, nb, BH, a.lag, quant, bh, j);
+      const int len = block_len(g, j);
+      const unsigned char* blk = sm_raw + b * buf_bytes;
+      if (!quant) {
+        const int cp = tid % npair, rg = tid / npair;
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(blk);
+        double s0 = 0.0, s1 = 0.0;
+        float mn0 = INFINITY, mn1 = INFINITY, mx0 = -INFINITY, mx1 = -INFINITY;
+        for (int o = rg; o < len; o += groups) {
+          const uint32_t v = w[o * npair + cp];
+          const float f0 = __uint_as_float(v << 16), f1 = __uint_as_float(v & 0xffff0000u);
+          s0 += static_cast<double>(f0);
+          s1 += static_cast<double>(f1);
+          mn0 = fminf(mn0, f0);
+          mn1 = fminf(mn1, f1);
+          mx0 = fmaxf(mx0, f0);
+          mx1 = fmaxf(mx1, f1);
+        }
+        dsum[rg * d + 2 * cp] = s0;
+        dsum[rg * d + 2 * cp + 1] = s1;
+        dmin[rg * d + 2 * cp] = mn0;
+        dmin[rg * d + 2 * cp + 1] = mn1;
+        dmax[rg * d + 2 * cp] = mx0;
+        dmax[rg * d + 2 * cp + 1] = mx1;
+        named_bar_sync(1, kSmoothThreads);
+        if (tid < d) {
+          double t = 0.0;
+          float vmin = INFINITY, vmax = -INFINITY;
+          for (int r = 0; r < groups; ++r) {
+            t += dsum[r * d + tid];
+            vmin = fminf(vmin, dmin[r * d + tid]);
+            vmax = fmaxf(vmax, dmax[r * d + tid]);
+          }
+          const float mu = static_cast<float>(t / static_cast<double>(len));
+          a.vmean[(static_cast<int64_t>(bh) * nb + j) * d + tid] = mu;
+          float am = fmaxf(0.f, fmaxf(vmax - mu, mu - vmin));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+          if (lane == 0) red[warp] = am;
+        }
+        named_bar_sync(1, kSmoothThreads);
+        if (tid == 0) {
+          float am = red[0];
+          for (int w2 = 1; w2 < d / 32; ++w2) am = fmaxf(am, red[w2]);
+          // non-negative floats order like their bit patterns
+          atomicMax(head_max + bh, __float_as_uint(am));
+          __threadfence();  // means and maximum before the count (after the barrier above)
+          atomicAdd(a.heads + bh, 1u);
+        }
+      } else {
+        const int e = slot[b].e;
+        if (tid == 0 && j == 0) a.vexp[bh] = e;
+        const float inv = ldexpf(1.0f, -e);  // exact power of two
+        const float2 inv2 = make_float2(inv, inv), nz2 = make_float2(-0.0f, -0.0f);
+        const float* mu = means + b * d;
+        uint8_t* dst = a.vq + (static_cast<int64_t>(bh) * nb + j) * d * g.bs;
+        for (int idx = tid; idx < nq * nrg; idx += kSmoothThreads) {
+          const int cq = idx % nq, rg = idx / nq;
+          const float4 m4 = *reinterpret_cast<const float4*>(mu + 4 * cq);
+          const float2 nm01 = make_float2(-m4.x, -m4.y), nm23 = make_float2(-m4.z, -m4.w);
+          uint32_t wc[4][4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            // rows rg*16 + 4q .. +3: x[u][c] for channel c of the quad
+            float x[4][4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int o = rg * 16 + 4 * q + u;
+              if (o < len) {
+                const uint2 v = *reinterpret_cast<const uint2*>(blk + (static_cast<size_t>(o) * d + 4 * cq) * 2);
+                // R = v - mu (fp32), then R * 2^-e (exact: -0 addend keeps signs)
+                const float2 r01 = ffma2(fadd2(make_float2(__uint_as_float(v.x << 16),
+                                                           __uint_as_float(v.x & 0xffff0000u)),
+                                               nm01),
+                                         inv2, nz2);
+                const float2 r23 = ffma2(fadd2(make_float2(__uint_as_float(v.y << 16),
+                                                           __uint_as_float(v.y & 0xffff0000u)),
+                                               nm23),
+                                         inv2, nz2);
+                x[u][0] = r01.x;
+                x[u][1] = r01.y;
+                x[u][2] = r23.x;
+                x[u][3] = r23.y;
+              } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) x[u][c] = 0.f;
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              wc[c][q] = e4m3x2(x[0][c], x[1][c]) | (e4m3x2(x[2][c], x[3][c]) << 16);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(4 * cq + c) * g.bs + rg * 16) =
+                make_uint4(wc[c][0], wc[c][1], wc[c][2], wc[c][3]);
+        }
+      }
+      // this warp is done with the buffer
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[b]));
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
     // the last CTA out resets the work counter and the head words
     __threadfence();
     const uint32_t prev = atomicAdd(&a.ctrl->aux_done, 1u);
@@ -297,7 +357,7 @@ cudaError_t launch_smooth_v(const sba_plan* p, const void* vt, void* vq, float* 
   a.heads = reinterpret_cast<uint32_t*>(ws + p->ws_heads);
   a.ctrl = reinterpret_cast<Ctrl*>(ws + p->ws_ctrl);
   a.budget_ns = p->wait_budget_ns;
-  const int smem = 2 * g.bs * g.d * 2;
+  const int smem = kSmoothBufs * (g.bs * g.d * 2 + g.d * 4);
   int dev = 0, sms = 0, per_sm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -306,22 +366,24 @@ cudaError_t launch_smooth_v(const sba_plan* p, const void* vt, void* vq, float* 
     e = cudaFuncSetAttribute(smooth_v_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
   }
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smooth_v_kernel, kSmoothThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smooth_v_kernel, kSmoothThreads + 32, smem);
   if (e != cudaSuccess) return e;
   // persistent: every CTA resident at once (a quantisation item waits on
   // statistics items that resident CTAs took earlier)
   const int64_t items = 2ll * g.B * g.H * g.nb;
   const int grid = static_cast<int>(std::min<int64_t>(items, static_cast<int64_t>(std::max(1, per_sm)) * sms));
   // Lag: the items taken between a head's last statistics item and its first
-  // quantisation item ((2L-1) nb) cover twice the items the CTAs hold (two
-  // each), so a quantisation item rarely waits; capped so that the lagged
-  // heads' values (L heads of nb blocks) stay within 48 MiB of L2.
+  // quantisation item ((2L-1) nb) cover twice the items the CTAs hold (a
+  // ring's worth and one more each), so a quantisation item rarely waits;
+  // capped so that the lagged heads' values (L heads of nb blocks) stay
+  // within 48 MiB of L2.
   const int64_t BH = static_cast<int64_t>(g.B) * g.H;
   const int64_t head_bytes = static_cast<int64_t>(g.nb) * g.bs * g.d * 2;
-  int64_t lag = ((4ll * grid + g.nb - 1) / g.nb + 2) / 2;
+  const int64_t held = static_cast<int64_t>(grid) * (kSmoothBufs + 1);
+  int64_t lag = ((2 * held + g.nb - 1) / g.nb + 2) / 2;
   lag = std::min(lag, std::max<int64_t>(1, (int64_t(48) << 20) / head_bytes));
   a.lag = static_cast<int>(std::max<int64_t>(1, std::min(lag, BH)));
-  smooth_v_kernel<<<grid, kSmoothThreads, smem, st>>>(g, a);
+  smooth_v_kernel<<<grid, kSmoothThreads + 32, smem, st>>>(g, a);
   return cudaGetLastError();
 }
 
