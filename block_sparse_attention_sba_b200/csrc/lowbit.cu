@@ -112,7 +112,9 @@ struct SmoothSlot {
 // fp32 (rounding is monotone, so the largest |fl(v - mu)| is at the largest
 // or the smallest v).
 // Quantisation item, one pass: thread = 4 channels x 16 rows; codes of one
-// channel's 16 rows are one 16-byte store.
+// channel's 16 rows are one 16-byte store. The consumer warps meet only inside
+// a statistics item (an mbarrier, bounded waits) and otherwise run through
+// the ring independently.
 __global__ void __launch_bounds__(kSmoothThreads + 32)
     smooth_v_kernel(KGeom g, SmoothArgs a) {
   extern __shared__ __align__(128) unsigned char sm_raw[];  // [bufs][bs][d] bf16, then [bufs][d] f32
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(kSmoothThreads + 32)
   __shared__ double dsum[512];                // [groups][d] partial sums
   __shared__ float dmin[512], dmax[512];      // [groups][d] partial minima / maxima
   __shared__ float red[kSmoothThreads / 32];
-  __shared__ __align__(8) uint64_t full[kSmoothBufs], empty[kSmoothBufs];
+  __shared__ __align__(8) uint64_t full[kSmoothBufs], empty[kSmoothBufs], sbar;
   __shared__ SmoothSlot slot[kSmoothBufs];
   __shared__ int s_abort;
   const int tid = threadIdx.x, d = g.d, nb = g.nb;
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(kSmoothThreads + 32)
       mbar_init(smem_u32(&full[b]), 1);
       mbar_init(smem_u32(&empty[b]), kSmoothThreads / 32);
     }
+    mbar_init(smem_u32(&sbar), kSmoothThreads);  // the consumers' own barrier
     fence_barrier_init();
     s_abort = 0;
   }
@@ -215,13 +218,22 @@ __global__ void __launch_bounds__(kSmoothThreads + 32)
     const int warp = tid >> 5, lane = tid & 31;
     const int npair = d / 2, groups = kSmoothThreads / npair;
     const int nq = d / 4, nrg = g.bs / 16;
+    uint32_t sph = 0;  // phases of sbar passed (the same count in every consumer)
+    // all consumers meet (bounded wait); false once the CTA aborts
+    auto consumers_meet = [&]() {
+      mbar_arrive(smem_u32(&sbar));
+      const bool ok = mbar_wait(smem_u32(&sbar), sph & 1u, a.budget_ns, abort_flag, status);
+      ++sph;
+      return ok;
+    };
     for (uint32_t k = 0;; ++k) {
       const int b = static_cast<int>(k % kSmoothBufs);
       const uint32_t use = k / kSmoothBufs;
+      // warps leave as a whole (lanes exchange values below); a warp that
+      // leaves after an abort ends the other consumers' waits through the
+      // abort flag, since every wait here is an mbarrier wait
       const bool got = mbar_wait(smem_u32(&full[b]), use & 1u, a.budget_ns, abort_flag, status);
-      // every consumer takes the same decision (the statistics path below
-      // has named barriers that need all of them)
-      if (named_bar_or(2, kSmoothThreads, !got || *abort_flag)) break;
+      if (__any_sync(0xffffffffu, !got)) break;
       const uint32_t item = slot[b].item;
       if (item >= n_items) break;
       bool quant;
@@ -250,7 +262,7 @@ __global__ void __launch_bounds__(kSmoothThreads + 32)
         dmin[rg * d + 2 * cp + 1] = mn1;
         dmax[rg * d + 2 * cp] = mx0;
         dmax[rg * d + 2 * cp + 1] = mx1;
-        named_bar_sync(1, kSmoothThreads);
+        if (__any_sync(0xffffffffu, !consumers_meet())) break;
         if (tid < d) {
           double t = 0.0;
           float vmin = INFINITY, vmax = -INFINITY;
@@ -266,7 +278,7 @@ __global__ void __launch_bounds__(kSmoothThreads + 32)
           for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
           if (lane == 0) red[warp] = am;
         }
-        named_bar_sync(1, kSmoothThreads);
+        if (__any_sync(0xffffffffu, !consumers_meet())) break;
         if (tid == 0) {
           float am = red[0];
           for (int w2 = 1; w2 < d / 32; ++w2) am = fmaxf(am, red[w2]);
