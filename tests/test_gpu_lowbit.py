@@ -209,3 +209,47 @@ def test_lowbit_hilbert_order_every_row():
     assert g.N % g.bs != 0  # the last block is partial
     blocks = [(0, h, i) for h in range(wl.H) for i in range(g.nb)]
     _check_attention(wl, gpu, codes, mu, e, blocks)
+
+
+@pytest.mark.parametrize("d,cube", [(64, (4, 4, 4)), (128, (4, 4, 4)), (64, (2, 8, 8))])
+def test_smooth_v_other_shapes_and_special_values(d, cube):
+    """sba_smooth_v on its own for the head and block sizes other than 128 x
+    128 (each takes its own thread mapping), bit-exact against the oracle,
+    on ragged grids with: a head whose values are all equal (every residual
+    0, so e = 0 and every code 0), and a head holding zeros, negative zeros,
+    bf16 subnormals and a few large values. A second call gives the same
+    bits (the kernel's counters reset themselves)."""
+    _need_gpu()
+    import block_sparse_attention_sba_b200 as sba
+    dev = torch.device("cuda:0")
+    B, H, T, Hh, W = 1, 3, 5, 9, 11
+    N = T * Hh * W
+    _, _, v = datagen.random_qkv(B, H, N, d, seed=7)
+    v = v.clone()
+    v[0, 1] = 0.375
+    rng = np.random.default_rng(11)
+    flat = v[0, 2].view(-1)
+    for val, n in ((0.0, 200), (-0.0, 200), (1e-40, 50), (-3e-39, 50), (300.0, 3)):
+        idx = torch.from_numpy(rng.choice(flat.numel(), n, replace=False))
+        flat[idx] = torch.tensor(val, dtype=torch.bfloat16)
+    v = v.to(dev)
+    plan = sba.Plan(B, H, T, Hh, W, d, cube, "bf16")
+    sa = sba.SparseAttention(plan, device=dev)
+    inf = plan.info
+    h = plan.handle
+    sba.sba_reorder(h, v, v, v, sa.qt, sa.kt, sa.vt, sa.workspace)
+    g = oracle.Geom(T, Hh, W, *cube)
+    codes, mu, e = oracle.v_smooth(to64(sa.vt.cpu()), g)
+    ref_q = codes.reshape(B, H, g.nb, g.bs, d).transpose(0, 1, 2, 4, 3)
+    assert e[0, 1] == 0 and not ref_q[0, 1].any()
+    assert e[0, 2] > e[0, 0]  # the large values set head 2's scale
+    for _ in range(2):
+        vq = torch.full((B, H, inf.nb, d, inf.bs), 0xAB, dtype=torch.uint8, device=dev)
+        vmean = torch.full((B, H, inf.nb, d), float("nan"), dtype=torch.float32, device=dev)
+        vexp = torch.full((B, H), -999, dtype=torch.int32, device=dev)
+        sba.sba_smooth_v(h, sa.vt, vq, vmean, vexp, sa.workspace)
+        torch.cuda.synchronize()
+        assert sa.check() == 0
+        assert np.array_equal(vexp.cpu().numpy().astype(np.int64), e)
+        assert np.array_equal(vmean.cpu().numpy(), mu)
+        assert np.array_equal(vq.cpu().numpy(), ref_q)
