@@ -48,7 +48,7 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sched-report", action="store_true")
     ap.add_argument("--no-lowbit", action="store_true", help="skip the low-bit P.V measurement")
-    ap.add_argument("--no-sweep", action="store_true", help="skip the Top-p 0.5 / 0.7 report")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the Top-p 0.4 / 0.5 / 0.7 report")
     ap.add_argument("--sched-workload", default="stress",
                     help="workload of the scheduler report (LPT persistent vs head-major grid)")
     ap.add_argument("--sched-reps", type=int, default=3, help="launches per schedule in that report")
@@ -547,7 +547,7 @@ def run_ours(args):
     sweep = None
     if not args.no_sweep and wl.name == "wan":
         sweep = []
-        for p_sw in (0.5, 0.7):
+        for p_sw in (0.4, 0.5, 0.7):
             tp = [p_sw] * wl.H
             t = {"reorder": [], "build_mask": [], "attention": [], "unreorder": []}
             for it in range(3 + 5):
