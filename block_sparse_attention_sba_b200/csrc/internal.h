@@ -17,7 +17,7 @@ struct sba_plan {
   size_t ws_qbar, ws_kbar; // offsets of the pooled means (fp64 [B*H][nb][d])
   size_t ws_scores, scores_bytes;  // pooled scores of a chunk of heads (fp64 [heads][nb][nb])
   size_t ws_perm;          // Hilbert order: offset of token_of_slot (int32 [Npad])
-  size_t ws_heads;         // per-(b, h) counters of sba_smooth_v (uint32 [B*H], zero between calls)
+  size_t ws_heads;         // sba_smooth_v per-(b, h) words: counts, then maxima (uint32 [2][B*H], zero between calls)
   uint64_t wait_budget_ns; // bounded-wait limit for device waits
   std::vector<int32_t> slot_of_token;  // Hilbert order: int32 [N]
   std::vector<int32_t> token_of_slot;  // Hilbert order: int32 [Npad], -1 = padding
