@@ -194,6 +194,17 @@ def max_over_ranks(value: float, pg, device="cpu") -> float:
     return float(t.item())
 
 
+def step_launches(B: int, H: int, nb: int) -> int:
+    """Kernel launches of one step: reorder, attention and unreorder once each,
+    and sba_build_mask's pooling, head scan and finalize once plus one score and
+    one cut launch per chunk of heads (the library forms the fp64 pooled scores
+    of as many heads at a time as 48 MiB hold, at least one)."""
+    per_head = nb * nb * 8
+    heads = max(1, max(per_head, 48 << 20) // per_head)
+    chunks = -(-(B * H) // min(heads, B * H))
+    return 3 + 3 + 2 * chunks
+
+
 def whole_job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
     """Weak scaling: every rank processes its own replica; the job's rate is
     all ranks' FLOPs over the slowest rank's time."""
@@ -604,7 +615,7 @@ def run_ours(args):
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": f_tile},
             "scheduler": sched, "lowbit": lowbit, "sparsity_sweep": sweep,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 7 * args.steps,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": step_launches(wl.B, wl.H, nb) * args.steps,
             "clocks": clocks, "device_status": sba.sba_status_string(status),
         }
         print(json.dumps(line), flush=True)
